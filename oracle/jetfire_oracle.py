@@ -1,0 +1,272 @@
+"""CPU oracle for the per-block (32x32) INT8 data flow of Jetfire.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import, call or execute this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` / ``--impl reference`` legs
+of ``bench.py`` use it. It shares no code with the CUDA library (``int8_fully_quantized_b200``)
+and imports nothing from it.
+
+What it computes, and where that comes from
+-------------------------------------------
+Source: "Jetfire: Efficient and Accurate Transformer Pretraining with INT8 Data Flow and
+Per-Block Quantization" (atlas.scime.ai summary page), section "Approach": every linear and
+non-linear operator reads and writes INT8 tensors that carry one scale factor per block, the
+block size is B = 32, quantization happens on-chip, and the weight gradient is also an INT8
+computation with per-block scales. The "Fp8 vs int8" page gives the signed INT8 range and the
+dequantization x = FP(q) * s.
+
+The pages state no formula for the scale, no rounding mode and no accumulation order. The
+readings taken here (each listed in the design doc):
+
+* square 32x32 blocks, scale s = absmax(block) / 127 in fp32 (IEEE division), no zero point;
+* q = clamp(rint(x / s), -127, 127): fp32 IEEE division, then round-half-to-even; -128 is never
+  produced; an all-zero block (or one whose s underflows to 0) gives s = 0 and q = 0;
+* linear layers: for every 32-wide block kappa of the contraction axis the integer partial sum
+  P = sum q_A * q_B is exact, it is multiplied by c = fp32(s_A * s_B) (one fp32 rounding), the
+  products are summed exactly enough (fp64, each c*P exact in fp64) and rounded once to fp32;
+  the fp32 result is then re-quantized per 32x32 block with the rule above;
+* GELU is the exact erf form 0.5 x (1 + erf(x / sqrt 2)), evaluated as 0.5 x erfc(-x / sqrt 2)
+  so that it keeps its relative accuracy for negative x; LayerNorm uses the biased variance
+  over the full row of the dequantized input, eps = 1e-5 by default, fp32 gamma and beta;
+  both are evaluated in fp64 and rounded once to fp32 before re-quantization.
+
+Every function below is pinned by tests in ``tests/test_oracle_pins.py`` against hand-worked
+values, closed forms, brute force in exact rational arithmetic, or independent library
+routines; none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import numpy as np
+
+BLOCK = 32
+QMAX = 127
+
+__all__ = [
+    "BLOCK", "QMAX", "bf16_bits_to_f32", "f32_to_bf16_bits", "quantize", "quantize_block",
+    "dequantize_block", "block_scale_grid", "linear_fwd", "linear_dgrad", "linear_wgrad",
+    "requantize", "gelu_i8", "layernorm_i8", "gelu_f64", "quantization_mse",
+]
+
+
+# --------------------------------------------------------------------------------------------
+# dtype helpers (exact definitions, no method arithmetic)
+# --------------------------------------------------------------------------------------------
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    """bf16 (as a uint16 bit pattern) -> fp32, exact: bf16 is the upper half of an fp32."""
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def f32_to_bf16_bits(y: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 with round-to-nearest-even on the dropped 16 bits (finite inputs)."""
+    u = np.ascontiguousarray(y, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    return ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
+
+
+# --------------------------------------------------------------------------------------------
+# a1: per-block quantization (Jetfire summary, "Approach": per-block scale factors, B = 32;
+#     "Fp8 vs int8" page: INT8 range -128..127, of which +-127 is used symmetrically)
+# --------------------------------------------------------------------------------------------
+def quantize(x: np.ndarray, block_rows: int, block_cols: int):
+    """Quantize fp32 ``x`` [R, C] with one scale per ``block_rows x block_cols`` block.
+
+    Returns (q int8 [R, C], s fp32 [R/block_rows, C/block_cols]). With 32x32 blocks this is the
+    Jetfire per-block quantizer; with (R, C) blocks it is per-tensor quantization, with (1, C)
+    per-token and with (R, 1) per-channel (the summary's ablation baselines)."""
+    x = np.asarray(x, dtype=np.float32)
+    R, C = x.shape
+    if R % block_rows or C % block_cols:
+        raise ValueError(f"shape {x.shape} is not a whole number of {block_rows}x{block_cols} blocks")
+    nbr, nbc = R // block_rows, C // block_cols
+    xb = x.reshape(nbr, block_rows, nbc, block_cols)
+    # absmax of each block: exact in fp32 (|.| and max do not round); -0.0 counts as 0
+    amax = np.abs(xb).max(axis=(1, 3)) if x.size else np.zeros((nbr, nbc), np.float32)
+    s = (amax.astype(np.float32) / np.float32(QMAX)).astype(np.float32)     # fp32 IEEE division
+    s4 = s[:, None, :, None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = (xb / s4).astype(np.float32)                                     # fp32 IEEE division
+    t = np.where(s4 == 0, np.float32(0), t)                                  # zero block -> q = 0
+    q = np.clip(np.rint(t), -QMAX, QMAX).astype(np.int8)                     # round half to even
+    return q.reshape(R, C), s
+
+
+def quantize_block(x: np.ndarray):
+    """Jetfire per-block quantizer: 32x32 blocks. Input fp32 (bf16/fp16 widened exactly first)."""
+    return quantize(x, BLOCK, BLOCK)
+
+
+def block_scale_grid(s: np.ndarray, block_rows: int = BLOCK, block_cols: int = BLOCK) -> np.ndarray:
+    """Expand a scale grid [R/br, C/bc] to one scale per element [R, C]."""
+    return np.repeat(np.repeat(np.asarray(s, np.float32), block_rows, axis=0), block_cols, axis=1)
+
+
+# --------------------------------------------------------------------------------------------
+# a2: dequantization x = FP(q) * s ("Fp8 vs int8" page)
+# --------------------------------------------------------------------------------------------
+def dequantize_block(q: np.ndarray, s: np.ndarray, out: str = "f32") -> np.ndarray:
+    """y = fp32(q) * s (one fp32 rounding), then round-to-nearest-even to the output dtype.
+
+    ``out``: "f32" (fp32 array), "bf16" (uint16 bit pattern) or "f16" (float16 array)."""
+    y = (np.asarray(q).astype(np.float32) * block_scale_grid(s)).astype(np.float32)
+    if out == "f32":
+        return y
+    if out == "bf16":
+        return f32_to_bf16_bits(y)
+    if out == "f16":
+        return y.astype(np.float16)
+    raise ValueError(out)
+
+
+# --------------------------------------------------------------------------------------------
+# a3-a5: the three INT8 GEMMs of a linear layer with per-block scales (Jetfire summary,
+#        "Approach": linear operators read/write INT8 + per-block scales; the weight gradient is
+#        also computed in INT8 with per-block scales).
+# --------------------------------------------------------------------------------------------
+def _blockscaled_sum(a_blocks, b_blocks, c_blocks):
+    """sum over contraction blocks kappa of c[kappa] * (a[kappa] @ b[kappa]^T).
+
+    a_blocks[kappa]: int8 [m, 32]; b_blocks[kappa]: int8 [n, 32];
+    c_blocks[kappa]: fp32 [m, n] (the scale product, already rounded to fp32).
+    The integer partial P = a @ b^T is computed as an fp64 matmul: every term and partial sum is
+    an integer of magnitude <= 32 * 127^2 < 2^53, so the result is exact. c * P is exact in fp64
+    (24 + 20 significant bits). The sum over kappa is fp64 and is rounded once to fp32."""
+    acc = None
+    for a, b, c in zip(a_blocks, b_blocks, c_blocks):
+        P = a.astype(np.float64) @ b.astype(np.float64).T
+        term = c.astype(np.float64) * P
+        acc = term if acc is None else acc + term
+    return acc.astype(np.float32)
+
+
+def _rows(blocks, n_blocks):
+    return range(n_blocks) if blocks is None else list(blocks)
+
+
+def linear_fwd(Xq, Xs, Wq, Ws, row_blocks=None, col_blocks=None):
+    """Forward Y = X W^T. X [M, K], W [N, K] -> fp32 Y [M, N] (or the sub-grid of output blocks
+    ``row_blocks x col_blocks``, returned as [len(rb)*32, len(cb)*32]).
+
+    Y[m, n] = sum_kappa fp32(sX[m/32, kappa] * sW[n/32, kappa]) * sum_{k in kappa} Xq[m,k] Wq[n,k]."""
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    rb = _rows(row_blocks, M // BLOCK)
+    cb = _rows(col_blocks, N // BLOCK)
+    rows = np.concatenate([np.arange(i * BLOCK, (i + 1) * BLOCK) for i in rb]) if len(rb) else np.arange(0)
+    cols = np.concatenate([np.arange(j * BLOCK, (j + 1) * BLOCK) for j in cb]) if len(cb) else np.arange(0)
+    a_blocks, b_blocks, c_blocks = [], [], []
+    for kap in range(K // BLOCK):
+        ks = slice(kap * BLOCK, (kap + 1) * BLOCK)
+        a_blocks.append(Xq[rows, ks])
+        b_blocks.append(Wq[cols, ks])
+        sa = np.repeat(Xs[list(rb), kap], BLOCK)          # per output row
+        sb = np.repeat(Ws[list(cb), kap], BLOCK)          # per output col
+        c_blocks.append((sa[:, None] * sb[None, :]).astype(np.float32))
+    if not a_blocks:
+        return np.zeros((len(rows), len(cols)), np.float32)
+    return _blockscaled_sum(a_blocks, b_blocks, c_blocks)
+
+
+def linear_dgrad(dYq, dYs, Wq, Ws, row_blocks=None, col_blocks=None):
+    """Input gradient dX = dY W. dY [M, N], W [N, K] -> fp32 dX [M, K].
+
+    dX[m, k] = sum_nu fp32(sdY[m/32, nu] * sW[nu, k/32]) * sum_{n in nu} dYq[m,n] Wq[n,k]."""
+    M, N = dYq.shape
+    K = Wq.shape[1]
+    rb = _rows(row_blocks, M // BLOCK)
+    cb = _rows(col_blocks, K // BLOCK)
+    rows = np.concatenate([np.arange(i * BLOCK, (i + 1) * BLOCK) for i in rb]) if len(rb) else np.arange(0)
+    cols = np.concatenate([np.arange(j * BLOCK, (j + 1) * BLOCK) for j in cb]) if len(cb) else np.arange(0)
+    a_blocks, b_blocks, c_blocks = [], [], []
+    for nu in range(N // BLOCK):
+        ns = slice(nu * BLOCK, (nu + 1) * BLOCK)
+        a_blocks.append(dYq[rows, ns])                    # [m, 32]
+        b_blocks.append(Wq[ns][:, cols].T)                # W[n in nu, k] -> [k, 32]
+        sa = np.repeat(dYs[list(rb), nu], BLOCK)
+        sb = np.repeat(Ws[nu, list(cb)], BLOCK)
+        c_blocks.append((sa[:, None] * sb[None, :]).astype(np.float32))
+    if not a_blocks:
+        return np.zeros((len(rows), len(cols)), np.float32)
+    return _blockscaled_sum(a_blocks, b_blocks, c_blocks)
+
+
+def linear_wgrad(dYq, dYs, Xq, Xs, row_blocks=None, col_blocks=None):
+    """Weight gradient dW = dY^T X. dY [M, N], X [M, K] -> fp32 dW [N, K].
+
+    dW[n, k] = sum_mu fp32(sdY[mu, n/32] * sX[mu, k/32]) * sum_{m in mu} dYq[m,n] Xq[m,k]."""
+    M, N = dYq.shape
+    K = Xq.shape[1]
+    rb = _rows(row_blocks, N // BLOCK)
+    cb = _rows(col_blocks, K // BLOCK)
+    rows = np.concatenate([np.arange(i * BLOCK, (i + 1) * BLOCK) for i in rb]) if len(rb) else np.arange(0)
+    cols = np.concatenate([np.arange(j * BLOCK, (j + 1) * BLOCK) for j in cb]) if len(cb) else np.arange(0)
+    a_blocks, b_blocks, c_blocks = [], [], []
+    for mu in range(M // BLOCK):
+        ms = slice(mu * BLOCK, (mu + 1) * BLOCK)
+        a_blocks.append(dYq[ms][:, rows].T)               # dY[m in mu, n] -> [n, 32]
+        b_blocks.append(Xq[ms][:, cols].T)                # X[m in mu, k]  -> [k, 32]
+        sa = np.repeat(dYs[mu, list(rb)], BLOCK)
+        sb = np.repeat(Xs[mu, list(cb)], BLOCK)
+        c_blocks.append((sa[:, None] * sb[None, :]).astype(np.float32))
+    if not a_blocks:
+        return np.zeros((len(rows), len(cols)), np.float32)
+    return _blockscaled_sum(a_blocks, b_blocks, c_blocks)
+
+
+def requantize(y: np.ndarray):
+    """On-chip re-quantization of an fp32 operator output: the per-block quantizer again."""
+    return quantize_block(y)
+
+
+# --------------------------------------------------------------------------------------------
+# a6, a7: non-linear operators on INT8 blocks (Jetfire summary, "Approach" and "Problem": the
+#         memory-bound non-linear operators also read and write INT8 + per-block scales)
+# --------------------------------------------------------------------------------------------
+def _erfc(x: np.ndarray) -> np.ndarray:
+    from scipy.special import erfc
+    return erfc(x)
+
+
+def gelu_f64(x: np.ndarray) -> np.ndarray:
+    """GELU(x) = x Phi(x) = 0.5 x (1 + erf(x / sqrt 2)) in fp64, evaluated as
+    0.5 x erfc(-x / sqrt 2) (the same function; 1 + erf cancels for very negative x)."""
+    x = np.asarray(x, dtype=np.float64)
+    return 0.5 * x * _erfc(-x / np.sqrt(2.0))
+
+
+def gelu_i8(q: np.ndarray, s: np.ndarray):
+    """INT8 in -> dequantize (fp32 q*s) -> GELU in fp64 -> round to fp32 -> per-block quantize.
+    Returns (q_out, s_out, y_f32)."""
+    x = (np.asarray(q).astype(np.float32) * block_scale_grid(s)).astype(np.float32)
+    y = gelu_f64(x).astype(np.float32)
+    qo, so = quantize_block(y)
+    return qo, so, y
+
+
+def layernorm_i8(q: np.ndarray, s: np.ndarray, gamma: np.ndarray, beta: np.ndarray,
+                 eps: float = 1e-5):
+    """INT8 in -> x = fp32 q*s -> per row: mean, biased variance over all H columns (fp64) ->
+    y = (x - mean) / sqrt(var + eps) * gamma + beta (fp64, rounded once to fp32) -> per-block
+    quantize. Returns (q_out, s_out, y_f32)."""
+    x = (np.asarray(q).astype(np.float32) * block_scale_grid(s)).astype(np.float64)
+    H = x.shape[1]
+    mu = x.sum(axis=1, keepdims=True) / H
+    var = ((x - mu) ** 2).sum(axis=1, keepdims=True) / H
+    y = (x - mu) / np.sqrt(var + np.float64(np.float32(eps))) * np.asarray(gamma, np.float64)[None, :] \
+        + np.asarray(beta, np.float64)[None, :]
+    y = y.astype(np.float32)
+    qo, so = quantize_block(y)
+    return qo, so, y
+
+
+# --------------------------------------------------------------------------------------------
+# quantization error of a granularity (Jetfire summary, "Measured effects": per-block vs
+# per-token and per-channel quantization error; "Experimental setup": quantization MSE)
+# --------------------------------------------------------------------------------------------
+def quantization_mse(x: np.ndarray, granularity: str) -> float:
+    """Mean squared error of quantize -> dequantize for one granularity:
+    "block" (32x32), "token" (one scale per row), "channel" (per column), "tensor"."""
+    x = np.asarray(x, np.float32)
+    R, C = x.shape
+    br, bc = {"block": (BLOCK, BLOCK), "token": (1, C), "channel": (R, 1), "tensor": (R, C)}[granularity]
+    q, s = quantize(x, br, bc)
+    xr = q.astype(np.float32).astype(np.float64) * block_scale_grid(s, br, bc).astype(np.float64)
+    return float(np.mean((xr - x.astype(np.float64)) ** 2))

@@ -1,0 +1,390 @@
+"""Pins of the CPU oracle to things other than itself (CPU only).
+
+Each test checks an oracle function against a hand-worked example (``tests/golden``), a
+closed form, an invariant, an independent library routine, or brute force in exact rational
+arithmetic, so that a dropped term, a wrong sign or index, or a transposed operand in the
+oracle fails at least one of them.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from inputs import synthetic as S
+
+
+def _golden(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------------------------------------
+# quantizer
+# ---------------------------------------------------------------------------------------------
+def test_quantize_hand_worked(golden_dir):
+    g = _golden(golden_dir, "quantize_hand.json")
+    for case in g["cases"]:
+        x = np.zeros((32, 32), np.float32)
+        x[0, :len(case["x"])] = np.array(case["x"], np.float32)
+        q, s = O.quantize_block(x)
+        assert s.shape == (1, 1)
+        assert s[0, 0] == np.float32(case["s"])
+        assert q[0, :len(case["q"])].tolist() == case["q"]
+        assert not q[1:].any() and not q[0, len(case["q"]):].any()
+
+
+def test_quantize_error_bound_brute_force():
+    rng = np.random.default_rng(3)
+    x = S.activation(rng, 96, 160, 5, 40.0)
+    q, s = O.quantize_block(x)
+    sf = O.block_scale_grid(s).astype(np.float64)
+    err = np.abs(x.astype(np.float64) - q.astype(np.float64) * sf)
+    # q = rint(fl(x/s)); |fl(x/s) - x/s| <= 2^-24 * 128, so |x - q s| <= s (1/2 + 2^-16)
+    assert np.all(err <= sf * (0.5 + 2.0 ** -16))
+    assert q.min() >= -127 and q.max() <= 127
+    # every block with a nonzero absmax reaches |q| = 127
+    qa = np.abs(q.astype(np.int32)).reshape(3, 32, 5, 32).max(axis=(1, 3))
+    assert np.all(qa[s > 0] == 127)
+
+
+def test_quantize_scale_grid_orientation():
+    """Block (I, J) gets absmax 127 * 2^(I - 2J): the scale grid must be exactly 2^(I - 2J),
+    which fails on any transposed or mis-reshaped block bookkeeping."""
+    rng = np.random.default_rng(4)
+    R, C = 4 * 32, 3 * 32
+    x = (rng.uniform(-1, 1, size=(R, C))).astype(np.float32)
+    expect = np.zeros((4, 3), np.float32)
+    for I in range(4):
+        for J in range(3):
+            e = I - 2 * J
+            blk = x[I * 32:(I + 1) * 32, J * 32:(J + 1) * 32]
+            blk *= np.float32(2.0 ** e)
+            r, c = rng.integers(0, 32, 2)
+            blk[r, c] = np.float32(-127.0 * 2.0 ** e if (I + J) % 2 else 127.0 * 2.0 ** e)
+            expect[I, J] = np.float32(2.0 ** e)
+    q, s = O.quantize_block(x)
+    assert np.array_equal(s, expect)
+    for I in range(4):
+        for J in range(3):
+            assert np.abs(q[I * 32:(I + 1) * 32, J * 32:(J + 1) * 32]).max() == 127
+
+
+def test_quantize_ties_round_half_even():
+    rng = np.random.default_rng(5)
+    for e in (-3, 0, 4):
+        x = S.tie_block(e, rng)
+        q, s = O.quantize_block(x)
+        assert s[0, 0] == np.float32(2.0 ** e)
+        exact = x.astype(np.float64) / 2.0 ** e           # exactly n + 0.5 (or 127 at [0,0])
+        ties = np.ones_like(q, dtype=bool)
+        ties[0, 0] = False
+        assert np.all(np.abs(q[ties] - exact[ties]) == 0.5)
+        assert np.all(q[ties] % 2 == 0)
+        assert q[0, 0] == 127
+
+
+def test_quantize_special_blocks():
+    b = S.adversarial_blocks()
+    q, s = O.quantize_block(b)
+    # 0: all zero
+    assert s[0, 0] == 0 and not q[:, 0:32].any()
+    # 1: single nonzero -> +-127 there, zero elsewhere
+    assert s[0, 1] == np.float32(np.float32(3.25) / np.float32(127))
+    assert q[7, 32 + 5] == -127 and np.count_nonzero(q[:, 32:64]) == 1
+    # 2: both +absmax and -absmax reach +-127
+    assert q[0, 64] == 127 and q[31, 95] == -127
+    # 4: -0.0 entries quantize to 0; absmax from the nonzeros
+    assert s[0, 4] == np.float32(np.float32(2e-3) / np.float32(127))
+    assert q[10, 128 + 20] == -127 and q[3, 128 + 4] == 64  # 1e-3 / (2e-3/127) = 63.5 -> 64 (fl)
+    # 5: subnormal scale 2^-140 is exact; q = the integers the block was built from
+    assert s[0, 5] == np.float32(2.0 ** -140)
+    blk = b[:, 160:192].astype(np.float64) / 2.0 ** -140
+    assert np.array_equal(q[:, 160:192].astype(np.float64), blk)
+    # 6: absmax = 2^-149 -> s = 2^-149 / 127 underflows to 0 -> q = 0
+    assert s[0, 6] == 0 and not q[:, 192:224].any()
+    # 7: identical entries -> all 127
+    assert np.all(q[:, 224:256] == 127)
+
+
+def test_quantize_per_tensor_limit():
+    """With a block as large as the tensor the quantizer is per-tensor quantization; when every
+    32x32 block holds the global absmax, the per-block result must equal it bit for bit."""
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((64, 96)).astype(np.float32)
+    g = np.float32(9.0)
+    for I in range(2):
+        for J in range(3):
+            x[I * 32 + (I * 7 + J) % 32, J * 32 + (3 * J + 1) % 32] = g if (I + J) % 2 == 0 else -g
+    qb, sb = O.quantize_block(x)
+    qt, st = O.quantize(x, 64, 96)
+    assert st.shape == (1, 1) and st[0, 0] == np.float32(g / np.float32(127))
+    assert np.all(sb == st[0, 0])
+    assert np.array_equal(qb, qt)
+
+
+def test_granularity_mse_direction():
+    """Jetfire summary, 'Measured effects': per-block quantization lowers the quantization error
+    versus per-token quantization on activations with channel-wise outliers (a direction pin)."""
+    rng = np.random.default_rng(0)
+    x = S.activation(rng, 512, 1024, 10, 30.0)
+    mb = O.quantization_mse(x, "block")
+    mt = O.quantization_mse(x, "token")
+    mT = O.quantization_mse(x, "tensor")
+    assert mb < mt <= mT * 1.0000001
+
+
+# ---------------------------------------------------------------------------------------------
+# dtype conversions and dequantize
+# ---------------------------------------------------------------------------------------------
+def test_bf16_conversions_match_torch():
+    rng = np.random.default_rng(7)
+    y = np.concatenate([rng.standard_normal(4096).astype(np.float32) * 100,
+                        np.array([0.0, -0.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 3.0e38, -1e-40], np.float32)])
+    ours = O.f32_to_bf16_bits(y)
+    ref = torch.from_numpy(y).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+    back = O.bf16_bits_to_f32(ours)
+    assert np.array_equal(back, torch.from_numpy(ref.view(np.int16)).view(torch.bfloat16).float().numpy())
+
+
+def test_dequantize_hand_and_round_trip():
+    q = np.zeros((32, 64), np.int8)
+    q[0, :4] = [1, -2, 127, -127]
+    q[5, 40] = 3
+    s = np.array([[0.5, 0.25]], np.float32)
+    y = O.dequantize_block(q, s)
+    assert y[0, :4].tolist() == [0.5, -1.0, 63.5, -63.5] and y[5, 40] == 0.75
+    assert np.count_nonzero(y) == 5
+    # values that are exactly q * 2^e come back exactly
+    rng = np.random.default_rng(8)
+    qi = rng.integers(-127, 128, size=(64, 64)).astype(np.int8)
+    qi[0, 0] = 127; qi[0, 32] = 127; qi[32, 0] = 127; qi[32, 32] = -127
+    x = qi.astype(np.float32) * np.float32(2.0 ** -5)
+    q2, s2 = O.quantize_block(x)
+    assert np.array_equal(O.dequantize_block(q2, s2), x)
+    # round trip error bound on random data
+    x = S.activation(rng, 64, 64, 2, 20.0)
+    q3, s3 = O.quantize_block(x)
+    err = np.abs(O.dequantize_block(q3, s3).astype(np.float64) - x)
+    assert np.all(err <= O.block_scale_grid(s3) * (0.5 + 2.0 ** -16) + 1e-30)
+    # bf16 / f16 outputs are the round-to-nearest-even of the fp32 result
+    yb = O.dequantize_block(q3, s3, "bf16")
+    assert np.array_equal(yb, torch.from_numpy(O.dequantize_block(q3, s3)).to(torch.bfloat16)
+                          .view(torch.int16).numpy().view(np.uint16))
+    assert np.array_equal(O.dequantize_block(q3, s3, "f16"),
+                          torch.from_numpy(O.dequantize_block(q3, s3)).half().numpy())
+
+
+# ---------------------------------------------------------------------------------------------
+# the three GEMMs
+# ---------------------------------------------------------------------------------------------
+def _const_blocks(scale, sign):
+    scale = np.asarray(scale, np.float32)
+    sign = np.asarray(sign, np.float32)
+    v = np.kron(sign * scale * np.float32(127), np.ones((32, 32), np.float32)).astype(np.float32)
+    return v
+
+
+def test_gemm_hand_worked_64(golden_dir):
+    g = _golden(golden_dir, "gemm_hand_64.json")
+    A = _const_blocks(g["A_scale"], g["A_sign"])
+    B = _const_blocks(g["B_scale"], g["B_sign"])
+    Aq, As = O.quantize_block(A)
+    Bq, Bs = O.quantize_block(B)
+    assert np.array_equal(As, np.array(g["A_scale"], np.float32))
+    assert np.all(np.abs(Aq) == 127)
+    outs = {
+        "fwd": O.linear_fwd(Aq, As, Bq, Bs),
+        "dgrad": O.linear_dgrad(Aq, As, Bq, Bs),
+        "wgrad": O.linear_wgrad(Aq, As, Bq, Bs),
+    }
+    for mode, y in outs.items():
+        exp = np.kron(np.array(g[mode]["Y"], np.float32), np.ones((32, 32), np.float32))
+        assert np.array_equal(y, exp), mode
+        q, s = O.requantize(y)
+        assert np.array_equal(s, np.array(g[mode]["s"], np.float32)), mode
+        assert np.array_equal(q, np.kron(np.array(g[mode]["q_sign"]) * 127, np.ones((32, 32))).astype(np.int8)), mode
+
+
+def _fp32_product(a, b):
+    """fp32(a*b) from the exact rational product: a*b of two fp32 values is exact in a double,
+    and one conversion to fp32 rounds it once."""
+    return Fraction(float(np.float32(float(Fraction(float(a)) * Fraction(float(b))))))
+
+
+@pytest.mark.parametrize("mode", ["fwd", "dgrad", "wgrad"])
+def test_gemm_exact_rational_brute_force(mode):
+    """Brute force with Python integers and Fractions, written from the definitions
+    Y = X W^T, dX = dY W, dW = dY^T X with one fp32 scale product per 32-block of the
+    contraction axis. The oracle's fp32 output must be the exact value rounded (within
+    0.5 ulp plus the fp64 summation slack)."""
+    rng = np.random.default_rng({"fwd": 10, "dgrad": 11, "wgrad": 12}[mode])
+    m, n, k = 64, 96, 96          # output rows, output cols, contraction
+    def qt(r, c):
+        q = rng.integers(-127, 128, size=(r, c)).astype(np.int8)
+        s = (rng.uniform(0.01, 2.0, size=(r // 32, c // 32))).astype(np.float32)
+        return q, s
+    if mode == "fwd":
+        Aq, As = qt(m, k); Bq, Bs = qt(n, k)
+        y = O.linear_fwd(Aq, As, Bq, Bs)
+        a = lambda i, kk: int(Aq[i, kk]); b = lambda j, kk: int(Bq[j, kk])
+        sa = lambda i, kap: As[i // 32, kap]; sb = lambda j, kap: Bs[j // 32, kap]
+    elif mode == "dgrad":          # A = dY [m, k], B = W [k, n]
+        Aq, As = qt(m, k); Bq, Bs = qt(k, n)
+        y = O.linear_dgrad(Aq, As, Bq, Bs)
+        a = lambda i, kk: int(Aq[i, kk]); b = lambda j, kk: int(Bq[kk, j])
+        sa = lambda i, kap: As[i // 32, kap]; sb = lambda j, kap: Bs[kap, j // 32]
+    else:                          # A = dY [k, m], B = X [k, n]
+        Aq, As = qt(k, m); Bq, Bs = qt(k, n)
+        y = O.linear_wgrad(Aq, As, Bq, Bs)
+        a = lambda i, kk: int(Aq[kk, i]); b = lambda j, kk: int(Bq[kk, j])
+        sa = lambda i, kap: As[kap, i // 32]; sb = lambda j, kap: Bs[kap, j // 32]
+    assert y.shape == (m, n)
+    for i in range(0, m, 7):
+        for j in range(0, n, 5):
+            exact = Fraction(0)
+            mag = Fraction(0)
+            for kap in range(k // 32):
+                P = sum(a(i, kk) * b(j, kk) for kk in range(kap * 32, kap * 32 + 32))
+                c = _fp32_product(sa(i, kap), sb(j, kap))
+                exact += c * P
+                mag += abs(c * P)
+            got = Fraction(float(y[i, j]))
+            ulp = Fraction(float(np.spacing(np.float32(abs(y[i, j])))))
+            assert abs(got - exact) <= ulp / 2 + mag * Fraction(1, 2 ** 45), (i, j)
+
+
+def test_gemm_power_of_two_scales_exact():
+    """All scales equal powers of two and small integer codes: every fp32 partial sum is exact,
+    so Y must equal the int64 matrix product times 2^e bit for bit."""
+    rng = np.random.default_rng(13)
+    M, K, N = 96, 256, 64
+    Xq = rng.integers(-15, 16, size=(M, K)).astype(np.int8)
+    Wq = rng.integers(-15, 16, size=(N, K)).astype(np.int8)
+    Xs = np.full((M // 32, K // 32), 2.0 ** -3, np.float32)
+    Ws = np.full((N // 32, K // 32), 2.0 ** -6, np.float32)
+    y = O.linear_fwd(Xq, Xs, Wq, Ws)
+    exact = (Xq.astype(np.int64) @ Wq.astype(np.int64).T).astype(np.float64) * 2.0 ** -9
+    assert np.array_equal(y.astype(np.float64), exact)
+    # per-K-block powers of two (different per block): still exact
+    Xs2 = (2.0 ** rng.integers(-4, 3, size=(M // 32, K // 32))).astype(np.float32)
+    y2 = O.linear_fwd(Xq, Xs2, Wq, Ws)
+    ex2 = np.zeros((M, N))
+    for kap in range(K // 32):
+        ks = slice(kap * 32, kap * 32 + 32)
+        P = Xq[:, ks].astype(np.int64) @ Wq[:, ks].astype(np.int64).T
+        ex2 += P * np.repeat(Xs2[:, kap].astype(np.float64), 32)[:, None] * 2.0 ** -6
+    assert np.array_equal(y2.astype(np.float64), ex2)
+
+
+def test_gemm_modes_are_transposes_of_each_other():
+    """dX = dY W is the forward product with W^T as the weight; dW = dY^T X is the forward
+    product of dY^T and X^T. Quantized blocks are square, so transposing a quantized tensor
+    transposes its codes and its scale grid. Checked bit for bit (catches index-map errors)."""
+    rng = np.random.default_rng(14)
+    M, N, K = 96, 64, 128
+    dYq, dYs = O.quantize_block(S.grad(rng, M, N))
+    Wq, Ws = O.quantize_block(S.weight(rng, N, K))
+    Xq, Xs = O.quantize_block(S.activation(rng, M, K, 2, 30.0))
+    assert np.array_equal(O.linear_dgrad(dYq, dYs, Wq, Ws), O.linear_fwd(dYq, dYs, Wq.T.copy(), Ws.T.copy()))
+    assert np.array_equal(O.linear_wgrad(dYq, dYs, Xq, Xs),
+                          O.linear_fwd(dYq.T.copy(), dYs.T.copy(), Xq.T.copy(), Xs.T.copy()))
+    # against a float64 matmul of the dequantized operands, when all scales of the contraction
+    # axis are equal (then the per-block rescale factors out of the sum)
+    Xs1 = np.repeat(Xs[:, :1], K // 32, axis=1)
+    Ws1 = np.repeat(Ws[:, :1], K // 32, axis=1)
+    ref = (Xq.astype(np.float64) * np.repeat(Xs1[:, 0], 32)[:, None]) @ \
+          (Wq.astype(np.float64) * np.repeat(Ws1[:, 0], 32)[:, None]).T
+    y = O.linear_fwd(Xq, Xs1, Wq, Ws1)
+    assert np.allclose(y, ref, rtol=2e-6, atol=1e-9 * np.abs(ref).max())
+
+
+def test_gemm_sampled_blocks_equal_full():
+    rng = np.random.default_rng(15)
+    M, N, K = 128, 96, 64
+    Xq, Xs = O.quantize_block(S.activation(rng, M, K, 1, 10.0))
+    Wq, Ws = O.quantize_block(S.weight(rng, N, K))
+    dYq, dYs = O.quantize_block(S.grad(rng, M, N))
+    full = O.linear_fwd(Xq, Xs, Wq, Ws)
+    part = O.linear_fwd(Xq, Xs, Wq, Ws, row_blocks=[3, 1], col_blocks=[2])
+    assert np.array_equal(part, np.concatenate([full[96:128, 64:96], full[32:64, 64:96]]))
+    full = O.linear_dgrad(dYq, dYs, Wq, Ws)
+    assert np.array_equal(O.linear_dgrad(dYq, dYs, Wq, Ws, [2], [0, 1]), full[64:96, 0:64])
+    full = O.linear_wgrad(dYq, dYs, Xq, Xs)
+    assert np.array_equal(O.linear_wgrad(dYq, dYs, Xq, Xs, [1], [1]), full[32:64, 32:64])
+
+
+# ---------------------------------------------------------------------------------------------
+# GELU_i8 and LayerNorm_i8
+# ---------------------------------------------------------------------------------------------
+def test_gelu_table_and_identities(golden_dir):
+    g = _golden(golden_dir, "normal_cdf_table.json")
+    x = np.array(g["x"])
+    assert np.allclose(O.gelu_f64(x), x * np.array(g["Phi"]), rtol=1e-15, atol=0)
+    from scipy.stats import norm
+    xs = np.linspace(-8, 8, 2001)
+    assert np.allclose(O.gelu_f64(xs), xs * norm.cdf(xs), rtol=1e-13, atol=1e-300)
+    # Phi(x) + Phi(-x) = 1  =>  GELU(x) - GELU(-x) = x
+    assert np.allclose(O.gelu_f64(xs) - O.gelu_f64(-xs), xs, rtol=0, atol=4e-15 * 8)
+    assert O.gelu_f64(np.array([0.0]))[0] == 0.0
+
+
+def test_gelu_i8_special_blocks():
+    # all-zero block -> zero output
+    q = np.zeros((32, 64), np.int8)
+    s = np.array([[0.0, 0.5]], np.float32)
+    qo, so, _ = O.gelu_i8(q, s)
+    assert so[0, 0] == 0 and so[0, 1] == 0 and not qo.any()
+    # a block of large positive values: GELU(x) = x in fp32 (Phi(x) = 1 - 1e-23), so the block
+    # re-quantizes to the same codes and (within an ulp) the same scale
+    rng = np.random.default_rng(16)
+    q = rng.integers(1, 128, size=(32, 32)).astype(np.int8)
+    q[0, 0] = 127
+    s = np.array([[0.5]], np.float32)                 # smallest value 0.5*1 ... too small; shift
+    x_min = 20.0
+    q = (q.astype(np.int32) // 2 + 64).astype(np.int8)   # codes 64..127
+    q[0, 0] = 127
+    s = np.array([[x_min / 64]], np.float32)
+    qo, so, y = O.gelu_i8(q, s)
+    assert np.array_equal(y, q.astype(np.float32) * s[0, 0])
+    assert np.array_equal(qo, q)
+    assert abs(float(so[0, 0]) - float(s[0, 0])) <= float(np.spacing(s[0, 0]))
+    # negative large values map to (nearly) 0: GELU(-20) ~ -5.5e-88 -> fp32 0
+    qo, so, y = O.gelu_i8(-q, s)
+    assert np.all(y == 0) and so[0, 0] == 0
+
+
+def test_layernorm_i8_vs_torch_and_invariants():
+    rng = np.random.default_rng(17)
+    M, H = 64, 256
+    x = S.activation(rng, M, H, 3, 50.0)
+    q, s = O.quantize_block(x)
+    gamma = rng.uniform(0.5, 1.5, H).astype(np.float32)
+    beta = rng.normal(0, 0.1, H).astype(np.float32)
+    qo, so, y = O.layernorm_i8(q, s, gamma, beta, 1e-5)
+    xd = torch.from_numpy((q.astype(np.float32) * O.block_scale_grid(s)).astype(np.float64))
+    ref = torch.nn.functional.layer_norm(xd, (H,), torch.from_numpy(gamma.astype(np.float64)),
+                                         torch.from_numpy(beta.astype(np.float64)),
+                                         eps=float(np.float32(1e-5))).numpy()
+    assert np.all(np.abs(y.astype(np.float64) - ref) <= np.abs(ref) * 2.0 ** -23 + 1e-12)
+    # requantization is the block quantizer of y
+    q2, s2 = O.quantize_block(y)
+    assert np.array_equal(q2, qo) and np.array_equal(s2, so)
+    # gamma = 1, beta = 0: rows have mean 0 and variance 1 (up to eps)
+    _, _, y1 = O.layernorm_i8(q, s, np.ones(H, np.float32), np.zeros(H, np.float32), 1e-5)
+    assert np.all(np.abs(y1.astype(np.float64).mean(axis=1)) < 1e-6)
+    assert np.all(np.abs(y1.astype(np.float64).var(axis=1) - 1) < 1e-4)
+    # scale invariance (eps = 0): doubling every block scale (exact) leaves y unchanged
+    _, _, ya = O.layernorm_i8(q, s, gamma, beta, 0.0)
+    _, _, yb = O.layernorm_i8(q, s * np.float32(2), gamma, beta, 0.0)
+    assert np.allclose(ya, yb, rtol=0, atol=2e-6 * np.abs(ya).max())
+    # a constant row gives y = beta exactly
+    qc = np.full((32, H), 5, np.int8)
+    sc = np.full((1, H // 32), 0.25, np.float32)
+    _, _, yc = O.layernorm_i8(qc, sc, gamma, beta, 1e-5)
+    assert np.array_equal(yc, np.broadcast_to(beta, yc.shape))
