@@ -1,0 +1,159 @@
+/*
+ * jetfire.h - C ABI of the per-block (32x32) INT8 data-flow library for B200 (sm_100a).
+ *
+ * What is computed (source: "Jetfire: Efficient and Accurate Transformer Pretraining with INT8
+ * Data Flow and Per-Block Quantization", atlas.scime.ai summary page, section "Approach"):
+ * every linear and non-linear operator of a transformer layer reads and writes INT8 tensors that
+ * carry one scale factor per block, with block size B = 32; quantization is applied on-chip, and
+ * the weight gradient is also computed in INT8 with per-block scales. The "Fp8 vs int8" page gives
+ * the signed INT8 range and the dequantization x = FP(q) * s.
+ *
+ * Readings taken where the pages are silent (each is stated once here and applies to every call):
+ *   - blocks are 32 x 32; block (I, J) covers rows 32I..32I+31 and columns 32J..32J+31;
+ *   - the scale of a block is s = absmax / 127 in fp32 (IEEE division, no zero point);
+ *   - a code is q = clamp(rint(x / s), -127, 127): IEEE fp32 quotient, round half to even;
+ *     -128 is never produced (it is accepted on input); an all-zero block, or one whose s
+ *     underflows to 0, gets s = 0 and codes 0; subnormals are honoured (no flush to zero);
+ *   - the GEMMs rescale the exact int32 partial of every 32-wide block of the contraction axis by
+ *     fp32(s_A * s_B) and accumulate in fp32 (block order unspecified), then re-quantize the fp32
+ *     result per 32x32 block on-chip;
+ *   - GELU is 0.5 x (1 + erf(x / sqrt 2)); LayerNorm uses the biased variance over the full row.
+ *
+ * Data layout (all device memory, all row-major and contiguous, all owned by the caller):
+ *   a quantized tensor T of shape [rows, cols] is a pair
+ *     T.q  int8  [rows, cols]          codes, 16-byte aligned
+ *     T.s  fp32  [rows/32, cols/32]    one scale per block, 4-byte aligned
+ *   rows and cols must be multiples of 32 (0 is allowed: the call does nothing).
+ *
+ * Execution: every call validates its arguments on the host, returns an error code without
+ * enqueuing anything if they are invalid, otherwise enqueues its kernel(s) on `stream` (a
+ * cudaStream_t passed as void*; NULL = the legacy default stream) and returns without waiting.
+ * The library never allocates, frees or retains device memory. Outputs must not overlap inputs.
+ * Inputs must be finite. Kernel-side failures (a bounded wait that timed out) are reported by
+ * jf_device_status(). Calls are thread-safe; calls on different streams may run concurrently.
+ * There is no CPU fallback: on a machine without an sm_100 GPU every compute call returns
+ * JF_ERR_DEVICE.
+ */
+#ifndef JETFIRE_H
+#define JETFIRE_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define JF_API __attribute__((visibility("default")))
+#else
+#define JF_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Read-only quantized tensor (device pointers). */
+typedef struct {
+  const int8_t* q;
+  const float* s;
+  int64_t rows, cols;
+} jf_cqtensor;
+
+/* Writable quantized tensor (device pointers). */
+typedef struct {
+  int8_t* q;
+  float* s;
+  int64_t rows, cols;
+} jf_qtensor;
+
+/* Element types of unquantized tensors. */
+typedef enum { JF_F32 = 0, JF_BF16 = 1, JF_F16 = 2 } jf_dtype;
+
+/* Status codes. */
+typedef enum {
+  JF_OK = 0,
+  JF_ERR_NULL = -1,    /* a required pointer is NULL */
+  JF_ERR_SHAPE = -2,   /* a dimension is negative, not a multiple of 32, or shapes disagree */
+  JF_ERR_ALIGN = -3,   /* a pointer is not aligned as documented */
+  JF_ERR_DTYPE = -4,   /* unknown jf_dtype */
+  JF_ERR_ALIAS = -5,   /* an output overlaps an input */
+  JF_ERR_CUDA = -6,    /* a CUDA runtime or driver call failed (launch, tensor-map encode) */
+  JF_ERR_TIMEOUT = -7, /* reported by jf_device_status: a kernel's bounded wait ran out */
+  JF_ERR_DEVICE = -8   /* no usable sm_100 device is current */
+} jf_status;
+
+/*
+ * a1. Per-block quantization (summary, "Approach": per-block scale factors, B = 32).
+ *   x     device, [rows, cols] row-major of dtype `dt` (fp32, bf16 or fp16), 16-byte aligned
+ *   q     device, int8 [rows, cols], 16-byte aligned (output)
+ *   s     device, fp32 [rows/32, cols/32], 4-byte aligned (output)
+ * Codes and scales are bit-exact with the rule above (bf16/fp16 are widened exactly first).
+ */
+JF_API int jf_quantize_block(const void* x, jf_dtype dt, int64_t rows, int64_t cols, int8_t* q, float* s,
+                      void* stream);
+
+/*
+ * a2. Dequantization y = fp32(q) * s, rounded to nearest even into `dt` ("Fp8 vs int8" page).
+ *   q, s  the quantized tensor (device, layout as above)
+ *   y     device, [rows, cols] of dtype `dt`, 16-byte aligned (output); bit-exact.
+ */
+JF_API int jf_dequantize_block(const int8_t* q, const float* s, int64_t rows, int64_t cols, void* y, jf_dtype dt,
+                        void* stream);
+
+/*
+ * a3. Linear forward Y = X W^T (summary, "Approach": INT8 linear operator with per-block scales).
+ *   X  [M, K] quantized activations, W [N, K] quantized weights, Y [M, N] (output).
+ *   Y(m, n) = sum_kb fp32(sX(m/32, kb) sW(n/32, kb)) * sum_{k in kb} Xq(m, k) Wq(n, k),
+ *   re-quantized per 32x32 block into Y.q / Y.s.
+ *   y_f32  optional device fp32 [M, N] (16-byte aligned) that receives the fp32 result before
+ *          re-quantization. Y.q may be NULL (then Y.s is ignored) when y_f32 is given; at least
+ *          one of the two outputs is required.
+ */
+JF_API int jf_linear_fwd(jf_cqtensor X, jf_cqtensor W, jf_qtensor Y, float* y_f32, void* stream);
+
+/*
+ * a4. Input gradient dX = dY W (the INT8 backward of the linear layer).
+ *   dY [M, N], W [N, K] (read re-blocked along N, no transpose pass), dX [M, K] (output).
+ *   dX(m, k) = sum_nb fp32(sdY(m/32, nb) sW(nb, k/32)) * sum_{n in nb} dYq(m, n) Wq(n, k).
+ *   dx_f32 as y_f32 above.
+ */
+JF_API int jf_linear_dgrad(jf_cqtensor dY, jf_cqtensor W, jf_qtensor dX, float* dx_f32, void* stream);
+
+/*
+ * a5. Weight gradient dW = dY^T X (summary, "Approach": "the weight gradient is also computed in
+ *     INT8 with per-block scales").
+ *   dY [M, N], X [M, K] (both read re-blocked along M), dW [N, K] (output).
+ *   dW(n, k) = sum_mb fp32(sdY(mb, n/32) sX(mb, k/32)) * sum_{m in mb} dYq(m, n) Xq(m, k).
+ *   dw_f32 as y_f32 above (an optimizer, or a data-parallel gradient reduction, wants fp32).
+ */
+JF_API int jf_linear_wgrad(jf_cqtensor dY, jf_cqtensor X, jf_qtensor dW, float* dw_f32, void* stream);
+
+/*
+ * a6. GELU on INT8 blocks (summary, "Approach" and "Problem": non-linear operators read and write
+ *     INT8 with per-block scales). Y = requant(GELU(fp32(X.q) * X.s)), same shape as X.
+ */
+JF_API int jf_gelu_i8(jf_cqtensor X, jf_qtensor Y, void* stream);
+
+/*
+ * a7. LayerNorm on INT8 blocks. Per row r of X [M, H]: x = fp32(q) * s, mean and biased variance
+ *     over the H columns, y = (x - mean) / sqrt(var + eps) * gamma + beta, re-quantized per block.
+ *   gamma, beta  device fp32 [H], 16-byte aligned.
+ */
+JF_API int jf_layernorm_i8(jf_cqtensor X, const float* gamma, const float* beta, float eps, jf_qtensor Y,
+                    void* stream);
+
+/* Static description of a status code (never NULL). */
+JF_API const char* jf_strerror(int status);
+
+/*
+ * Synchronizes `stream`, then returns and clears the device-side status of the library on the
+ * current device: JF_OK, or JF_ERR_TIMEOUT if a kernel gave up a bounded wait since the last
+ * call (its outputs are then undefined), or JF_ERR_CUDA if the synchronization failed.
+ */
+JF_API int jf_device_status(void* stream);
+
+/* Number of SMs of the current device, as the kernels size their grids (0 if none). */
+JF_API int jf_sm_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JETFIRE_H */

@@ -1,0 +1,255 @@
+// C ABI of the library: argument validation, then the kernel launch (see include/jetfire.h).
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "jetfire.h"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace jf {
+__device__ unsigned int g_status = 0u;
+}
+
+namespace {
+
+struct DevInfo {
+  int sm_count = 0;
+  bool ok = false;
+  unsigned int* status = nullptr;  // device address of jf::g_status on this device
+};
+
+// Per-device SM count and capability check (cached per device ordinal).
+DevInfo device_info() {
+  static DevInfo cache[64];
+  static bool probed[64] = {false};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return DevInfo{};
+  }
+  if (!probed[dev]) {
+    DevInfo d;
+    int major = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) {
+      d.ok = (major == 10);
+      d.sm_count = sms;
+      void* addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, jf::g_status) == cudaSuccess) {
+        d.status = static_cast<unsigned int*>(addr);
+      } else {
+        cudaGetLastError();
+        d.ok = false;
+      }
+    } else {
+      cudaGetLastError();
+    }
+    cache[dev] = d;
+    probed[dev] = true;
+  }
+  return cache[dev];
+}
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+inline bool dims_ok(int64_t r, int64_t c) {
+  return r >= 0 && c >= 0 && (r % 32) == 0 && (c % 32) == 0 && r < (int64_t(1) << 31) && c < (int64_t(1) << 31);
+}
+inline bool overlap(const void* a, int64_t na, const void* b, int64_t nb) {
+  if (a == nullptr || b == nullptr || na <= 0 || nb <= 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + uintptr_t(nb) && b0 < a0 + uintptr_t(na);
+}
+inline int64_t elem_size(jf_dtype dt) { return dt == JF_F32 ? 4 : 2; }
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? JF_OK : JF_ERR_CUDA; }
+
+int check_cq(const jf_cqtensor& t) {
+  if (!dims_ok(t.rows, t.cols)) return JF_ERR_SHAPE;
+  if (t.rows == 0 || t.cols == 0) return JF_OK;
+  if (t.q == nullptr || t.s == nullptr) return JF_ERR_NULL;
+  if (!aligned(t.q, 16) || !aligned(t.s, 4)) return JF_ERR_ALIGN;
+  return JF_OK;
+}
+
+// Output quantized tensor; `need_q` false allows q == NULL (fp32-only output).
+int check_q(const jf_qtensor& t, bool need_q) {
+  if (!dims_ok(t.rows, t.cols)) return JF_ERR_SHAPE;
+  if (t.rows == 0 || t.cols == 0) return JF_OK;
+  if (t.q == nullptr) return need_q ? JF_ERR_NULL : JF_OK;
+  if (t.s == nullptr) return JF_ERR_NULL;
+  if (!aligned(t.q, 16) || !aligned(t.s, 4)) return JF_ERR_ALIGN;
+  return JF_OK;
+}
+
+int64_t qbytes(const jf_cqtensor& t) { return t.rows * t.cols; }
+int64_t sbytes(int64_t r, int64_t c) { return (r / 32) * (c / 32) * 4; }
+
+// Shared validation + launch of the three GEMMs. A/B are the stored operands.
+int gemm_call(int mode, const jf_cqtensor& A, const jf_cqtensor& B, const jf_qtensor& Y, float* y_f32,
+              int64_t rows, int64_t cols, int64_t depth, void* stream) {
+  int st;
+  if ((st = check_cq(A)) != JF_OK) return st;
+  if ((st = check_cq(B)) != JF_OK) return st;
+  if ((st = check_q(Y, false)) != JF_OK) return st;
+  if (Y.rows != rows || Y.cols != cols) return JF_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return JF_OK;
+  if (Y.q == nullptr && y_f32 == nullptr) return JF_ERR_NULL;
+  if (y_f32 != nullptr && !aligned(y_f32, 16)) return JF_ERR_ALIGN;
+  // outputs must not overlap inputs (nor each other)
+  const void* ins[4] = {A.q, A.s, B.q, B.s};
+  const int64_t in_n[4] = {qbytes(A), sbytes(A.rows, A.cols), qbytes(B), sbytes(B.rows, B.cols)};
+  const void* outs[3] = {Y.q, Y.q ? Y.s : nullptr, y_f32};
+  const int64_t out_n[3] = {rows * cols, sbytes(rows, cols), rows * cols * 4};
+  for (int o = 0; o < 3; ++o) {
+    for (int i = 0; i < 4; ++i)
+      if (overlap(outs[o], out_n[o], ins[i], in_n[i])) return JF_ERR_ALIAS;
+    for (int o2 = o + 1; o2 < 3; ++o2)
+      if (overlap(outs[o], out_n[o], outs[o2], out_n[o2])) return JF_ERR_ALIAS;
+  }
+  const DevInfo d = device_info();
+  if (!d.ok) return JF_ERR_DEVICE;
+  jf::GemmArgs g;
+  g.mode = mode;
+  g.a_q = A.q;
+  g.a_s = A.s;
+  g.b_q = B.q;
+  g.b_s = B.s;
+  g.rows = rows;
+  g.cols = cols;
+  g.depth = depth;
+  g.a_ld = A.cols;
+  g.b_ld = B.cols;
+  g.y_q = Y.q;
+  g.y_s = Y.q ? Y.s : nullptr;
+  g.y_f32 = y_f32;
+  g.status = d.status;
+  if (depth == 0) {
+    // empty contraction: the result is exactly zero (codes 0, scales 0)
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    if (Y.q) {
+      e = cudaMemsetAsync(Y.q, 0, size_t(rows * cols), s);
+      if (e == cudaSuccess) e = cudaMemsetAsync(Y.s, 0, size_t(sbytes(rows, cols)), s);
+    }
+    if (e == cudaSuccess && y_f32) e = cudaMemsetAsync(y_f32, 0, size_t(rows * cols * 4), s);
+    return cuda_status(e);
+  }
+  return cuda_status(jf::launch_gemm(g, d.sm_count, static_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+int jf_quantize_block(const void* x, jf_dtype dt, int64_t rows, int64_t cols, int8_t* q, float* s,
+                      void* stream) {
+  if (dt != JF_F32 && dt != JF_BF16 && dt != JF_F16) return JF_ERR_DTYPE;
+  if (!dims_ok(rows, cols)) return JF_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return JF_OK;
+  if (x == nullptr || q == nullptr || s == nullptr) return JF_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(s, 4)) return JF_ERR_ALIGN;
+  const int64_t nx = rows * cols * elem_size(dt);
+  if (overlap(q, rows * cols, x, nx) || overlap(s, sbytes(rows, cols), x, nx) ||
+      overlap(q, rows * cols, s, sbytes(rows, cols)))
+    return JF_ERR_ALIAS;
+  const DevInfo d = device_info();
+  if (!d.ok) return JF_ERR_DEVICE;
+  return cuda_status(jf::launch_quantize(x, int(dt), rows, cols, q, s, d.sm_count, static_cast<cudaStream_t>(stream)));
+}
+
+int jf_dequantize_block(const int8_t* q, const float* s, int64_t rows, int64_t cols, void* y, jf_dtype dt,
+                        void* stream) {
+  if (dt != JF_F32 && dt != JF_BF16 && dt != JF_F16) return JF_ERR_DTYPE;
+  if (!dims_ok(rows, cols)) return JF_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return JF_OK;
+  if (q == nullptr || s == nullptr || y == nullptr) return JF_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(s, 4) || !aligned(y, 16)) return JF_ERR_ALIGN;
+  const int64_t ny = rows * cols * elem_size(dt);
+  if (overlap(y, ny, q, rows * cols) || overlap(y, ny, s, sbytes(rows, cols))) return JF_ERR_ALIAS;
+  const DevInfo d = device_info();
+  if (!d.ok) return JF_ERR_DEVICE;
+  return cuda_status(jf::launch_dequantize(q, s, rows, cols, y, int(dt), d.sm_count, static_cast<cudaStream_t>(stream)));
+}
+
+int jf_linear_fwd(jf_cqtensor X, jf_cqtensor W, jf_qtensor Y, float* y_f32, void* stream) {
+  if (!dims_ok(X.rows, X.cols) || !dims_ok(W.rows, W.cols)) return JF_ERR_SHAPE;
+  if (X.cols != W.cols) return JF_ERR_SHAPE;
+  return gemm_call(jf::kFwd, X, W, Y, y_f32, X.rows, W.rows, X.cols, stream);
+}
+
+int jf_linear_dgrad(jf_cqtensor dY, jf_cqtensor W, jf_qtensor dX, float* dx_f32, void* stream) {
+  if (!dims_ok(dY.rows, dY.cols) || !dims_ok(W.rows, W.cols)) return JF_ERR_SHAPE;
+  if (dY.cols != W.rows) return JF_ERR_SHAPE;
+  return gemm_call(jf::kDgrad, dY, W, dX, dx_f32, dY.rows, W.cols, dY.cols, stream);
+}
+
+int jf_linear_wgrad(jf_cqtensor dY, jf_cqtensor X, jf_qtensor dW, float* dw_f32, void* stream) {
+  if (!dims_ok(dY.rows, dY.cols) || !dims_ok(X.rows, X.cols)) return JF_ERR_SHAPE;
+  if (dY.rows != X.rows) return JF_ERR_SHAPE;
+  return gemm_call(jf::kWgrad, dY, X, dW, dw_f32, dY.cols, X.cols, dY.rows, stream);
+}
+
+int jf_gelu_i8(jf_cqtensor X, jf_qtensor Y, void* stream) {
+  int st;
+  if ((st = check_cq(X)) != JF_OK) return st;
+  if ((st = check_q(Y, true)) != JF_OK) return st;
+  if (X.rows != Y.rows || X.cols != Y.cols) return JF_ERR_SHAPE;
+  if (X.rows == 0 || X.cols == 0) return JF_OK;
+  const int64_t nq = qbytes(X), ns = sbytes(X.rows, X.cols);
+  if (overlap(Y.q, nq, X.q, nq) || overlap(Y.q, nq, X.s, ns) || overlap(Y.s, ns, X.q, nq) ||
+      overlap(Y.s, ns, X.s, ns) || overlap(Y.q, nq, Y.s, ns))
+    return JF_ERR_ALIAS;
+  const DevInfo d = device_info();
+  if (!d.ok) return JF_ERR_DEVICE;
+  return cuda_status(jf::launch_gelu_i8(X.q, X.s, X.rows, X.cols, Y.q, Y.s, d.sm_count, static_cast<cudaStream_t>(stream)));
+}
+
+int jf_layernorm_i8(jf_cqtensor X, const float* gamma, const float* beta, float eps, jf_qtensor Y,
+                    void* stream) {
+  int st;
+  if ((st = check_cq(X)) != JF_OK) return st;
+  if ((st = check_q(Y, true)) != JF_OK) return st;
+  if (X.rows != Y.rows || X.cols != Y.cols) return JF_ERR_SHAPE;
+  if (X.rows == 0 || X.cols == 0) return JF_OK;
+  if (gamma == nullptr || beta == nullptr) return JF_ERR_NULL;
+  if (!aligned(gamma, 16) || !aligned(beta, 16)) return JF_ERR_ALIGN;
+  const int64_t nq = qbytes(X), ns = sbytes(X.rows, X.cols);
+  if (overlap(Y.q, nq, X.q, nq) || overlap(Y.q, nq, X.s, ns) || overlap(Y.s, ns, X.q, nq) ||
+      overlap(Y.s, ns, X.s, ns) || overlap(Y.q, nq, Y.s, ns) || overlap(Y.q, nq, gamma, X.cols * 4) ||
+      overlap(Y.q, nq, beta, X.cols * 4) || overlap(Y.s, ns, gamma, X.cols * 4) || overlap(Y.s, ns, beta, X.cols * 4))
+    return JF_ERR_ALIAS;
+  const DevInfo d = device_info();
+  if (!d.ok) return JF_ERR_DEVICE;
+  return cuda_status(
+      jf::launch_layernorm_i8(X.q, X.s, X.rows, X.cols, gamma, beta, eps, Y.q, Y.s, static_cast<cudaStream_t>(stream)));
+}
+
+const char* jf_strerror(int status) {
+  switch (status) {
+    case JF_OK: return "ok";
+    case JF_ERR_NULL: return "a required pointer is NULL";
+    case JF_ERR_SHAPE: return "bad shape: dimensions must be non-negative multiples of 32 and agree";
+    case JF_ERR_ALIGN: return "misaligned pointer (codes and fp32/bf16/fp16 data: 16 bytes; scales: 4 bytes)";
+    case JF_ERR_DTYPE: return "unknown dtype";
+    case JF_ERR_ALIAS: return "an output overlaps an input or another output";
+    case JF_ERR_CUDA: return "a CUDA runtime/driver call failed";
+    case JF_ERR_TIMEOUT: return "a kernel's bounded wait timed out; outputs are undefined";
+    case JF_ERR_DEVICE: return "no usable sm_100 (B200) device is current";
+    default: return "unknown status";
+  }
+}
+
+int jf_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return JF_ERR_CUDA;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, jf::g_status, sizeof(v)) != cudaSuccess) return JF_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(jf::g_status, &zero, sizeof(zero)) != cudaSuccess) return JF_ERR_CUDA;
+  if (v & jf::kStatusTimeout) return JF_ERR_TIMEOUT;
+  return v ? JF_ERR_CUDA : JF_OK;
+}
+
+int jf_sm_count(void) {
+  const DevInfo d = device_info();
+  return d.sm_count;
+}
+
+}  // extern "C"

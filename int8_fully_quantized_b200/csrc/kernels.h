@@ -1,0 +1,39 @@
+// Internal launch functions (called by the C ABI in api.cu after argument validation).
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace jf {
+
+cudaError_t launch_quantize(const void* x, int dtype, int64_t R, int64_t C, int8_t* q, float* s, int sm_count,
+                            cudaStream_t st);
+cudaError_t launch_dequantize(const int8_t* q, const float* s, int64_t R, int64_t C, void* y, int dtype,
+                              int sm_count, cudaStream_t st);
+cudaError_t launch_gelu_i8(const int8_t* q, const float* s, int64_t R, int64_t C, int8_t* qo, float* so,
+                           int sm_count, cudaStream_t st);
+cudaError_t launch_layernorm_i8(const int8_t* q, const float* s, int64_t R, int64_t H, const float* gamma,
+                                const float* beta, float eps, int8_t* qo, float* so, cudaStream_t st);
+
+// Block-scaled INT8 GEMM: out[r, c] = sum over 32-blocks kb of the contraction axis of
+// fp32(sA(r/32, kb) * sB(c/32, kb)) * sum_{k in kb} A(r, k) B(c, k), re-quantized per 32x32 block.
+// The operand views differ per mode (see gemm.cu).
+enum GemmMode { kFwd = 0, kDgrad = 1, kWgrad = 2 };
+
+struct GemmArgs {
+  int mode;
+  const int8_t* a_q;  // A codes (X for fwd, dY for dgrad and wgrad)
+  const float* a_s;
+  const int8_t* b_q;  // B codes (W for fwd and dgrad, X for wgrad)
+  const float* b_s;
+  int64_t rows, cols, depth;  // output rows, output cols, contraction length
+  int64_t a_ld, b_ld;         // row pitch (elements) of the stored A and B matrices
+  int8_t* y_q;                // nullable
+  float* y_s;                 // non-null when y_q is
+  float* y_f32;               // nullable
+  unsigned int* status;       // device status word (bit flags of ptx.cuh)
+};
+
+cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t st);
+
+}  // namespace jf

@@ -1,0 +1,72 @@
+// Device-side per-block quantization rule shared by every kernel that emits INT8 blocks.
+//
+// Jetfire (atlas.scime.ai summary, "Approach"): INT8 tensors carry one scale per 32x32 block and
+// (re)quantization happens on-chip. Reading taken for the unstated formula: s = absmax / 127
+// (fp32 IEEE division), code = clamp(rint_half_even(x / s), -127, 127) with x / s the IEEE fp32
+// quotient, an all-zero block (or one whose s underflows to 0) gives s = 0 and codes 0.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+namespace jf {
+
+constexpr float kQMax = 127.0f;
+// 1.5 * 2^23. For |t| < 2^22, t + kRoundMagic (one fp32 rounding) is 1.5*2^23 + n with n the
+// integer nearest to t, ties to even, and the low byte of its bit pattern is n mod 256.
+constexpr float kRoundMagic = 12582912.0f;
+constexpr float kFltMinNormal = 1.17549435082228750797e-38f;
+
+struct BlockQuant {
+  float s;    // block scale
+  float inv;  // RN(1 / s); only used when s is a normal number
+  int mode;   // 0: s == 0, every code 0; 1: s subnormal, exact division everywhere; 2: fast path
+};
+
+__device__ __forceinline__ BlockQuant block_quant(float amax) {
+  BlockQuant b;
+  b.s = __fdiv_rn(amax, kQMax);
+  b.inv = __frcp_rn(b.s);
+  b.mode = (b.s == 0.0f) ? 0 : (b.s < kFltMinNormal ? 1 : 2);
+  return b;
+}
+
+// The low byte of the result is the INT8 code of x in a block quantized with b.
+//
+// Fast path (s normal): t = RN(x * RN(1/s)). With e = x/s exact and |e| <= 127 (1 + 2^-23),
+// |t - e| <= |e| (2^-23 + 2^-48) < 2^-16 and the IEEE quotient RN(e) is within 2^-18 of e, so
+// t and RN(e) differ by less than 2^-15. When t lies farther than 2^-14 from every half-integer,
+// both round to the same integer; otherwise (near a tie) the IEEE quotient is computed.
+__device__ __forceinline__ uint32_t quant_byte(float x, const BlockQuant& b) {
+  if (b.mode == 2) {
+    const float t = x * b.inv;
+    const float tp = t + kRoundMagic;
+    const float r = tp - kRoundMagic;
+    if (fabsf(t - r) < 0.49993896484375f) return __float_as_uint(tp);  // 0.5 - 2^-14
+  } else if (b.mode == 0) {
+    return 0u;
+  }
+  float t = __fdiv_rn(x, b.s);
+  t = fminf(fmaxf(t, -kQMax), kQMax);
+  return __float_as_uint(t + kRoundMagic);
+}
+
+// Pack the low bytes of four words into one word (a in byte 0 ... d in byte 3).
+__device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// Four signed INT8 codes (bytes of w) -> four exact fp32 values. Flipping the sign bit gives
+// q + 128 as an unsigned byte u; the fp32 with bit pattern 0x4B0000uu is 2^23 + u exactly.
+__device__ __forceinline__ void i8x4_to_f32(uint32_t w, float (&f)[4]) {
+  const uint32_t u = w ^ 0x80808080u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) f[i] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7440 | i)) - 8388736.0f;
+}
+
+// Largest of 32 non-negative floats across the warp (non-negative floats order like their bits).
+__device__ __forceinline__ float warp_max_nonneg(float m) {
+  return __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(m)));
+}
+
+}  // namespace jf

@@ -1,0 +1,94 @@
+"""C ABI checks that need no GPU: the library loads, exports every function declared in
+include/jetfire.h, and rejects invalid arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import int8_fully_quantized_b200 as jf
+from int8_fully_quantized_b200 import build_lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_lib.build()
+    return jf.load_library()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "jetfire.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:JF_API\s+)?(?:int|const char\s*\*)\s+(jf_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared()
+    for n in ("jf_quantize_block", "jf_dequantize_block", "jf_linear_fwd", "jf_linear_dgrad",
+              "jf_linear_wgrad", "jf_gelu_i8", "jf_layernorm_i8", "jf_strerror", "jf_device_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", build_lib.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\s[T]\s+(\w+)$", out, flags=re.M))
+    for name in _declared():
+        assert name in exported, name
+        assert hasattr(lib, name)
+    # nothing else of the library leaks out as a C symbol
+    assert sorted(n for n in exported if n.startswith("jf_")) == _declared()
+    assert set(jf.EXPORTED_SYMBOLS) == set(_declared())
+
+
+def test_strerror_is_total(lib):
+    for st in range(-10, 2):
+        assert isinstance(jf.jf_strerror(st), str) and jf.jf_strerror(st)
+
+
+def test_host_validation_rejects_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)           # 16-byte aligned, never dereferenced: validation fails first
+    odd = vp((1 << 20) + 4)
+    # shapes must be multiples of 32
+    assert lib.jf_quantize_block(fake, 1, 33, 64, fake, fake, None) == -2
+    assert lib.jf_quantize_block(fake, 1, -32, 64, fake, fake, None) == -2
+    # unknown dtype
+    assert lib.jf_quantize_block(fake, 7, 32, 32, fake, fake, None) == -4
+    # NULL pointers
+    assert lib.jf_quantize_block(None, 1, 32, 32, fake, fake, None) == -1
+    # misaligned codes
+    assert lib.jf_quantize_block(fake, 1, 32, 32, odd, vp((1 << 21)), None) == -3
+    # output overlapping the input
+    assert lib.jf_quantize_block(fake, 0, 32, 32, vp((1 << 20) + 64), vp(1 << 22), None) == -5
+    # empty tensors are a no-op
+    assert lib.jf_quantize_block(None, 1, 0, 64, None, None, None) == 0
+    # GEMM shape mismatch: X [64, 96] vs W [32, 64]
+    X = jf._CQ(1 << 20, 1 << 22, 64, 96)
+    W = jf._CQ(1 << 24, 1 << 26, 32, 64)
+    Y = jf._Q(1 << 28, 1 << 30, 64, 32)
+    assert lib.jf_linear_fwd(X, W, Y, None, None) == -2
+    # GEMM output shape must be [M, N]
+    W = jf._CQ(1 << 24, 1 << 26, 32, 96)
+    assert lib.jf_linear_fwd(X, W, jf._Q(1 << 28, 1 << 30, 64, 64), None, None) == -2
+    # no output at all
+    assert lib.jf_linear_fwd(X, W, jf._Q(None, None, 64, 32), None, None) == -1
+    # dgrad: dY [M, N] with W [N, K]; wgrad: dY [M, N] with X [M, K]
+    assert lib.jf_linear_dgrad(jf._CQ(1 << 20, 1 << 22, 64, 96), jf._CQ(1 << 24, 1 << 26, 64, 32),
+                               jf._Q(1 << 28, 1 << 30, 64, 32), None, None) == -2
+    assert lib.jf_linear_wgrad(jf._CQ(1 << 20, 1 << 22, 64, 96), jf._CQ(1 << 24, 1 << 26, 96, 32),
+                               jf._Q(1 << 28, 1 << 30, 96, 32), None, None) == -2
+    # LayerNorm needs gamma/beta
+    assert lib.jf_layernorm_i8(jf._CQ(1 << 20, 1 << 22, 32, 64), None, fake, ctypes.c_float(1e-5),
+                               jf._Q(1 << 28, 1 << 30, 32, 64), None) == -1
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_compute_without_gpu_fails_loudly(lib):
+    vp = ctypes.c_void_p
+    # valid arguments, but no sm_100 device is current: the call must refuse, never fall back
+    st = lib.jf_quantize_block(vp(1 << 20), 1, 32, 32, vp(1 << 24), vp(1 << 26), None)
+    assert st == -8
+    with pytest.raises(jf.JetfireError):
+        jf._check(st, "jf_quantize_block")
