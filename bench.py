@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""Benchmark of the per-block INT8 data-flow hot path on B200.
+
+One step = one pass of every operator of the path over one batch of the GPT2-medium MLP linear
+workload (tokens M = 4096, hidden K = 1024, N = 4096; X ~ N(0,1) with 1% of the channels x30,
+W ~ N(0, 0.02), dY ~ N(0, 1e-3), bf16 on entry):
+
+    quantize X -> LayerNorm_i8 -> quantize W -> linear fwd (Y = X W^T) -> GELU_i8
+    quantize dY -> dgrad (dX = dY W) -> wgrad (dW = dY^T X) -> dequantize dX to bf16
+
+Inputs are resident in HBM when the timed region starts; L2 is flushed between steps (a 256 MiB
+write outside the timed events). ``value`` is the whole-step throughput in TOPS counted on the
+three GEMMs (3 x 2MNK int8 ops per step and rank) over the step time, summed over ranks.
+``--gpus N`` (under torchrun) runs N data-parallel ranks, each with its own M = 4096 tokens; the
+fp32 weight-gradient partials are summed with NCCL and re-quantized (weak scaling).
+
+``--impl reference`` times the CPU oracle (the method written out plainly in numpy) on a bounded
+token sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "per-block INT8 GEMM TOPS (% INT8 peak); quantize/GELU/LN GB/s (% HBM)"
+WORKLOAD = "gpt2m_fc1"
+NOMINAL_I8_OVER_BF16 = 2.0       # dense int8 (4.5 POPS) / dense bf16 (2.25 PFLOP/s), nominal B200
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    p.add_argument("--cpu-sample-tokens", type=int, default=1024)
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only; nothing is changed)
+# --------------------------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap",
+               0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = None
+            try:
+                import torch
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            except Exception:
+                pass
+            h = None
+            if uuid:
+                for i in range(pynvml.nvmlDeviceGetCount()):
+                    hh = pynvml.nvmlDeviceGetHandleByIndex(i)
+                    u = pynvml.nvmlDeviceGetUUID(hh)
+                    u = u.decode() if isinstance(u, bytes) else u
+                    if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                        h = hh
+            self.h = h if h is not None else pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nvml = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - only without NVML
+            self.nvml = None
+            self.error = str(e)
+
+    def _run(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM))
+                mask = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if self.nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "error", "")}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples),
+                "window": "warm-up and timed steps, NVML every 5 ms"}
+
+
+# --------------------------------------------------------------------------------------------
+# host inputs
+# --------------------------------------------------------------------------------------------
+def host_inputs(M, K, N, seed_tokens, seed_weight):
+    from inputs import synthetic as S
+    w = S.WORKLOADS[WORKLOAD]
+    rng = np.random.default_rng(seed_tokens)
+    n_out, fac = w["x_outliers"]
+    x = S.activation(rng, M, K, n_out, fac)
+    dy = S.grad(rng, M, N)
+    wt = S.weight(np.random.default_rng(seed_weight), N, K)
+    rng_ln = np.random.default_rng(seed_weight + 7)
+    gamma = rng_ln.uniform(0.5, 1.5, K).astype(np.float32)
+    beta = rng_ln.normal(0, 0.1, K).astype(np.float32)
+    return {"x": S.to_bf16_bits(x), "w": S.to_bf16_bits(wt), "dy": S.to_bf16_bits(dy), "gamma": gamma, "beta": beta}
+
+
+def bytes_quant(r, c, in_bytes):  # read input, write codes + scales
+    return r * c * (in_bytes + 1) + (r // 32) * (c // 32) * 4
+
+
+def bytes_i8_op(r, c, extra=0):  # read codes + scales, write codes + scales
+    return 2 * (r * c + (r // 32) * (c // 32) * 4) + extra
+
+
+# --------------------------------------------------------------------------------------------
+# our implementation
+# --------------------------------------------------------------------------------------------
+class GpuStep:
+    OPS = ["quantize_x", "layernorm_i8", "quantize_w", "linear_fwd", "gelu_i8", "quantize_dy",
+           "linear_dgrad", "linear_wgrad", "dequantize_dx"]
+
+    def __init__(self, M, K, N, host, world_size):
+        import torch
+        import int8_fully_quantized_b200 as jf
+        self.jf, self.torch = jf, torch
+        self.M, self.K, self.N, self.world = M, K, N, world_size
+        dev = torch.device("cuda", torch.cuda.current_device())
+        bf = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        self.xb, self.wb, self.dyb = bf(host["x"]), bf(host["w"]), bf(host["dy"])
+        self.gamma = torch.from_numpy(host["gamma"]).to(dev)
+        self.beta = torch.from_numpy(host["beta"]).to(dev)
+        e = lambda r, c: jf.empty_qtensor(r, c, dev)
+        self.Xq, self.Xn, self.Wq, self.Y, self.G = e(M, K), e(M, K), e(N, K), e(M, N), e(M, N)
+        self.dYq, self.dX, self.dW = e(M, N), e(M, K), e(N, K)
+        self.dx_bf16 = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+        self.dw_f32 = torch.empty((N, K), dtype=torch.float32, device=dev) if world_size > 1 else None
+        self.launches_per_step = 9 + (1 if world_size > 1 else 0)
+        self.bytes = {
+            "quantize_x": bytes_quant(M, K, 2), "quantize_w": bytes_quant(N, K, 2), "quantize_dy": bytes_quant(M, N, 2),
+            "layernorm_i8": bytes_i8_op(M, K, 8 * K), "gelu_i8": bytes_i8_op(M, N),
+            "dequantize_dx": M * K * 3 + (M // 32) * (K // 32) * 4,
+        }
+        self.ops = {"linear_fwd": 2 * M * N * K, "linear_dgrad": 2 * M * K * N, "linear_wgrad": 2 * N * K * M}
+
+    def run(self, ev=None):
+        jf, t = self.jf, self.torch
+        mark = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
+        mark(0)
+        jf.jf_quantize_block(self.xb, self.Xq.q, self.Xq.s)
+        mark(1)
+        jf.jf_layernorm_i8(self.Xq, self.gamma, self.beta, 1e-5, self.Xn)
+        mark(2)
+        jf.jf_quantize_block(self.wb, self.Wq.q, self.Wq.s)
+        mark(3)
+        jf.jf_linear_fwd(self.Xn, self.Wq, self.Y, None)
+        mark(4)
+        jf.jf_gelu_i8(self.Y, self.G)
+        mark(5)
+        jf.jf_quantize_block(self.dyb, self.dYq.q, self.dYq.s)
+        mark(6)
+        jf.jf_linear_dgrad(self.dYq, self.Wq, self.dX, None)
+        mark(7)
+        if self.world > 1:
+            from int8_fully_quantized_b200.parallel import allreduce_wgrad_
+            jf.jf_linear_wgrad(self.dYq, self.Xn, None, self.dw_f32)
+            allreduce_wgrad_(self.dw_f32)
+            jf.jf_quantize_block(self.dw_f32, self.dW.q, self.dW.s)
+        else:
+            jf.jf_linear_wgrad(self.dYq, self.Xn, self.dW, None)
+        mark(8)
+        jf.jf_dequantize_block(self.dX.q, self.dX.s, self.dx_bf16)
+        mark(9)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import int8_fully_quantized_b200 as jf
+    from int8_fully_quantized_b200 import parallel as P
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    jf.load_library()
+    wl = __import__("inputs.synthetic", fromlist=["WORKLOADS"]).WORKLOADS[WORKLOAD]
+    M, K, N = wl["M"], wl["K"], wl["N"]
+    host = host_inputs(M, K, N, P.shard_seed(0, rank), seed_weight=0)
+    step = GpuStep(M, K, N, host, world)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")   # 256 MiB > L2
+    stream = torch.cuda.current_stream()
+
+    sampler = ClockSampler(local)
+    with sampler:
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            step.run()
+        st = jf.jf_device_status()
+        if st != 0:
+            raise RuntimeError(f"device status after warm-up: {jf.jf_strerror(st)}")
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(10)] for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.zero_()
+            step.run(evs[i])
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+    st = jf.jf_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after the timed steps: {jf.jf_strerror(st)}")
+    per_op = {op: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)]
+              for j, op in enumerate(GpuStep.OPS)}
+    step_ms_local = sum(evs[i][0].elapsed_time(evs[i][9]) for i in range(args.steps)) / args.steps
+    step_ms = P.max_over_ranks(step_ms_local, device="cuda")
+    ops_per_step = sum(step.ops.values())
+    value = world * ops_per_step / (step_ms * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    i8_peak_burst = peaks["bf16_tflops"] * NOMINAL_I8_OVER_BF16
+    kernels = {}
+    for op, ts in per_op.items():
+        ms = statistics.mean(ts)
+        if op in step.ops:
+            tops = step.ops[op] / (ms * 1e-3) / 1e12
+            kernels[op] = {"ms": round(ms, 4), "TOPS": round(tops, 1), "frac_i8_peak": round(tops / i8_peak_burst, 4)}
+        else:
+            gbs = step.bytes[op] / (ms * 1e-3) / 1e9
+            kernels[op] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+    gemm_ops = [op for op in step.ops]
+    dom = max(gemm_ops, key=lambda o: statistics.mean(per_op[o]))
+    dom_ms = statistics.mean(per_op[dom])
+    achieved = step.ops[dom] / (dom_ms * 1e-3) / 1e12
+    traffic = _load_traffic(dom)
+    roofline = {"kernel": f"gemm_i8_kernel ({dom})", "bound": "tensor", "achieved": round(achieved, 1),
+                "peak": round(i8_peak_burst, 1), "unit": "TOPS", "frac": round(achieved / i8_peak_burst, 4),
+                "traffic": traffic,
+                "peak_source": f"{peak_src} bf16 dense burst x {NOMINAL_I8_OVER_BF16:g} (nominal int8/bf16 ratio)",
+                "algorithmic": f"2*M*N*K = {step.ops[dom]} int8 ops per launch"}
+
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": round(step_ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
+        "config": {"workload": "GPT2-medium MLP fc1 linear fwd+dgrad+wgrad with quantize, LayerNorm_i8, GELU_i8 "
+                               "and dequantize (per rank)", "M": M, "K": K, "N": N, "block": 32,
+                   "inputs": "bf16 X ~N(0,1) with 10 channels x30, W ~N(0,0.02), dY ~N(0,1e-3)",
+                   "parallelism": f"dp{world}", "l2": "flushed between steps (256 MiB write, outside timed events)"},
+        "kernels": kernels, "roofline": roofline,
+        "gpu_launches": step.launches_per_step * args.steps,
+        "clocks": sampler.summary(),
+    }
+    if not args.no_e2e:
+        result["e2e"] = run_e2e(step, host, args, world, flush)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline(args.cpu_sample_tokens, host)
+        print(json.dumps(result), flush=True)
+
+
+def _load_traffic(kernel_op):
+    """dram read + write bytes per launch of the dominant kernel from the committed ncu summary
+    (profiles/gemm_traffic.json), or None when no capture of the current kernel exists."""
+    path = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        v = d.get(kernel_op)
+        return None if v is None else int(v)
+    except Exception:
+        return None
+
+
+def run_e2e(step, host, args, world, flush):
+    """Same step through the public API with host buffers: per step, pinned host -> device copies
+    of X, W and dY, the nine operators, and device -> host reads of dX (bf16) and dW (codes and
+    scales)."""
+    import torch
+    from int8_fully_quantized_b200 import parallel as P
+    pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hx, hw, hdy = pin(host["x"]), pin(host["w"]), pin(host["dy"])
+    out_dx = torch.empty(step.dx_bf16.shape, dtype=torch.bfloat16).pin_memory()
+    out_wq = torch.empty(step.dW.q.shape, dtype=torch.int8).pin_memory()
+    out_ws = torch.empty(step.dW.s.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hx, hw, hdy))
+    d2h = sum(t.numel() * t.element_size() for t in (out_dx, out_wq, out_ws))
+
+    def one(ev0=None, ev1=None):
+        if ev0 is not None:
+            ev0.record()
+        step.xb.copy_(hx, non_blocking=True)
+        step.wb.copy_(hw, non_blocking=True)
+        step.dyb.copy_(hdy, non_blocking=True)
+        step.run()
+        out_dx.copy_(step.dx_bf16, non_blocking=True)
+        out_wq.copy_(step.dW.q, non_blocking=True)
+        out_ws.copy_(step.dW.s, non_blocking=True)
+        if ev1 is not None:
+            ev1.record()
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        one()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        one(*evs[i])
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    ms = P.max_over_ranks(ms, device="cuda")
+    ops = sum(step.ops.values())
+    return {"value": round(world * ops / (ms * 1e-3) / 1e12, 2), "unit": "TOPS", "ms_per_step": round(ms, 4),
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+# --------------------------------------------------------------------------------------------
+# CPU oracle timings (the baseline leg, and the --impl reference arm)
+# --------------------------------------------------------------------------------------------
+def _oracle_step(host, tokens):
+    """The whole step in the CPU oracle on the first `tokens` tokens of the batch (W in full).
+    Returns the GEMM int8 ops it performed."""
+    import oracle as O
+    K = host["x"].shape[1]
+    N = host["w"].shape[0]
+    x = O.bf16_bits_to_f32(host["x"][:tokens])
+    w = O.bf16_bits_to_f32(host["w"])
+    dy = O.bf16_bits_to_f32(host["dy"][:tokens])
+    Xq, Xs = O.quantize_block(x)
+    Xn_q, Xn_s, _ = O.layernorm_i8(Xq, Xs, host["gamma"], host["beta"], 1e-5)
+    Wq, Ws = O.quantize_block(w)
+    Y = O.linear_fwd(Xn_q, Xn_s, Wq, Ws)
+    Yq, Ys = O.requantize(Y)
+    O.gelu_i8(Yq, Ys)
+    dYq, dYs = O.quantize_block(dy)
+    dX = O.linear_dgrad(dYq, dYs, Wq, Ws)
+    dXq, dXs = O.requantize(dX)
+    O.requantize(O.linear_wgrad(dYq, dYs, Xn_q, Xn_s))
+    O.dequantize_block(dXq, dXs, "bf16")
+    return 3 * 2 * tokens * N * K
+
+
+def _cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(tokens, host):
+    t0 = time.perf_counter()
+    ops = _oracle_step(host, tokens)
+    dt = time.perf_counter() - t0
+    return {"value": round(ops / dt / 1e12, 6), "unit": "TOPS", "cores": _cpu_cores(), "kind": "oracle",
+            "seconds": round(dt, 2),
+            "sample": f"one oracle step on the first {tokens} of the 4096 tokens (full W), GEMM int8 ops / wall time"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = __import__("inputs.synthetic", fromlist=["WORKLOADS"]).WORKLOADS[WORKLOAD]
+    M, K, N = wl["M"], wl["K"], wl["N"]
+    host = host_inputs(M, K, N, 1, seed_weight=0)
+    tokens = 256
+    for _ in range(max(3, args.warmup)):
+        _oracle_step(host, tokens)
+    times = []
+    ops = 0
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        ops = _oracle_step(host, tokens)
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * sum(times) / len(times)
+    value = ops / (ms * 1e-3) / 1e12
+    cores = _cpu_cores()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
+        "config": {"workload": "GPT2-medium MLP fc1 linear fwd+dgrad+wgrad with quantize, LayerNorm_i8, GELU_i8 "
+                               "and dequantize", "M": M, "K": K, "N": N, "block": 32, "parallelism": "oracle on host"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: the oracle's full step on the first {tokens} of the {M} tokens"},
+        "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

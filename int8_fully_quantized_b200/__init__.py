@@ -18,6 +18,7 @@ from typing import NamedTuple, Optional
 
 import torch
 
+from . import build_lib
 from .build_lib import LIB_PATH
 
 __all__ = [
@@ -61,6 +62,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     path = path or os.environ.get("JETFIRE_LIB", LIB_PATH)
     if not os.path.exists(path):
         raise RuntimeError(f"{path} is missing: build it with `python -m int8_fully_quantized_b200.build_lib`")
+    if path == LIB_PATH and not build_lib.up_to_date():
+        raise RuntimeError(f"{path} was not built from the current sources: rebuild it with "
+                           "`python -m int8_fully_quantized_b200.build_lib`")
     lib = ctypes.CDLL(path)
     vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
     lib.jf_quantize_block.argtypes = [vp, i32, i64, i64, vp, vp, vp]

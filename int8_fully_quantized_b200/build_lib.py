@@ -7,6 +7,7 @@ quantizer relies on IEEE division, reciprocal and denormal handling.
 from __future__ import annotations
 
 import glob
+import hashlib
 import os
 import shutil
 import subprocess
@@ -17,6 +18,7 @@ ROOT = os.path.dirname(PKG_DIR)
 CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libjetfire.so")
+HASH_PATH = LIB_PATH + ".srchash"
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
@@ -39,11 +41,26 @@ def _inputs() -> list[str]:
         glob.glob(os.path.join(INCLUDE, "*.h")) + [os.path.abspath(__file__)]
 
 
+def source_hash() -> str:
+    """Content hash of every file the library is built from (sources, headers, this script)."""
+    h = hashlib.sha256()
+    for p in sorted(_inputs()):
+        h.update(os.path.relpath(p, ROOT).encode())
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def built_hash() -> str | None:
+    try:
+        with open(HASH_PATH) as f:
+            return f.read().strip()
+    except OSError:
+        return None
+
+
 def up_to_date() -> bool:
-    if not os.path.exists(LIB_PATH):
-        return False
-    t = os.path.getmtime(LIB_PATH)
-    return all(os.path.getmtime(p) <= t for p in _inputs())
+    return os.path.exists(LIB_PATH) and built_hash() == source_hash()
 
 
 def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None) -> str:
@@ -61,6 +78,8 @@ def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | N
     if verbose and (res.stdout or res.stderr):
         print(res.stdout + res.stderr, file=sys.stderr)
     os.replace(tmp, LIB_PATH)
+    with open(HASH_PATH, "w") as f:
+        f.write(source_hash())
     return LIB_PATH
 
 

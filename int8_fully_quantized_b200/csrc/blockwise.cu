@@ -93,7 +93,7 @@ __device__ __forceinline__ void quant_pack(const float* v, const BlockQuant& b, 
 // block rows (full 32-byte sectors).
 // ---------------------------------------------------------------------------------------------
 template <typename T>
-__global__ void __launch_bounds__(256) quantize_kernel(const T* __restrict__ x, int64_t R, int64_t C,
+__global__ void __launch_bounds__(256, 4) quantize_kernel(const T* __restrict__ x, int64_t R, int64_t C,
                                                        int8_t* __restrict__ q, float* __restrict__ s) {
   constexpr int EPV = Vec<T>::kElems;      // elements per 16-byte vector
   constexpr int VPR = 32 / EPV;            // vectors per block row
@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(const T* __restrict__ x, 
 // (by output vectors).
 // ---------------------------------------------------------------------------------------------
 template <typename T>
-__global__ void __launch_bounds__(256) dequantize_kernel(const int8_t* __restrict__ q, const float* __restrict__ s,
+__global__ void __launch_bounds__(256, 4) dequantize_kernel(const int8_t* __restrict__ q, const float* __restrict__ s,
                                                          int64_t R, int64_t C, T* __restrict__ y) {
   constexpr int EPV = Vec<T>::kElems;
   constexpr int VPR = 32 / EPV;
@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const int8_t* __restric
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ float gelu_f32(float x) { return 0.5f * x * erfcf(x * -0.70710678118654752440f); }
 
-__global__ void __launch_bounds__(256) gelu_i8_kernel(const int8_t* __restrict__ q, const float* __restrict__ s,
+__global__ void __launch_bounds__(256, 4) gelu_i8_kernel(const int8_t* __restrict__ q, const float* __restrict__ s,
                                                       int64_t R, int64_t C, int8_t* __restrict__ qo,
                                                       float* __restrict__ so) {
   const int lane = threadIdx.x & 31;

@@ -7,18 +7,24 @@
 // exact int32 partial P = sum_k A(r,k) B(c,k) is multiplied by c = fp32(sA(r/32,kb) * sB(c/32,kb))
 // and accumulated in fp32; after the last block the fp32 tile is re-quantized per 32x32 block.
 //
-// Design (one CTA per SM, persistent over 128 x 256 output tiles):
-//   warp 0      TMA producer: 128-byte-deep stages of A (128 rows) and B (256 rows) into a
-//               4-stage shared-memory ring (128-byte swizzle), plus the 48 scales of the stage into
-//               a scale ring (cp.async).
-//   warp 1      TMEM allocator and MMA issuer: one tcgen05.mma (M=128, N=256, K=32) per 32-wide
-//               contraction block, each into a fresh int32 accumulator; two 256-column TMEM
-//               accumulators alternate so the MMA of block kb+1 overlaps the drain of block kb.
-//   warps 2-9   epilogue: warp w owns TMEM lanes 32 (w % 4) .. +31 (one 32-row block of the tile)
-//               and one 128-column half. Per contraction block it loads its int32 partials
-//               (tcgen05.ld), converts them and does acc = fma(c, P, acc) in registers. After the
-//               last block it reduces each 32x32 block's absmax across the warp and writes codes,
-//               the block scale and (optionally) the fp32 result.
+// Design (one CTA per SM, persistent over 128 x 128 output tiles). Every barrier operation, TMA
+// issue and commit costs its issuing thread a few hundred cycles of latency, so the three pipeline
+// roles run in separate warps and overlap:
+//   warp 0       producer: lane 0 loads 128-byte-deep stages of A and B (TMA, 128-byte swizzle)
+//                into a 6-stage shared-memory ring; all 32 lanes copy the stage's 32 scales into
+//                the same slot (cp.async). A slot is refilled once the epilogue has finished the
+//                stage it held, which also means the MMAs that read it have completed.
+//   warp 1       MMA: lane 0 issues one tcgen05.mma (M=128, N=128, K=32) per 32-wide contraction
+//                block, each into a fresh int32 accumulator. The four 128-column TMEM accumulators
+//                form two groups of two: the MMAs of a group share one tcgen05.commit (each commit
+//                drains the tensor pipe) and the two groups double-buffer against the epilogue.
+//                Warp 1 also owns TMEM.
+//   warps 2-17   epilogue: warp w owns TMEM lanes 32 (w % 4) .. +31 and one 32-column block, i.e.
+//                exactly one 32x32 output block of the tile; four warps per SM sub-partition hide
+//                each other's TMEM load latency. Per contraction block a warp loads its 32 int32
+//                partials per thread (tcgen05.ld), converts them and accumulates fp32(sA*sB) * P in
+//                registers. After the last block it reduces the block's absmax across the warp and
+//                writes the 32x32 codes, the block scale and (optionally) the fp32 result.
 // Operand orientation: A and B are read K-major (contraction contiguous) or MN-major (output
 // index contiguous) straight from their row-major INT8 storage, so dgrad and wgrad re-block along
 // the other axis with no transpose pass.
@@ -36,23 +42,23 @@
 namespace jf {
 
 constexpr int BM = 128;             // tile rows = MMA M = TMEM lanes
-constexpr int BN = 256;             // tile cols = MMA N
+constexpr int BN = 128;             // tile cols = MMA N
 constexpr int KB = 32;              // contraction block (one MMA, one rescale)
 constexpr int KBS = 4;              // contraction blocks per pipeline stage (128 bytes)
-constexpr int STAGES = 4;
-constexpr int SC_SLOTS = 8;
-constexpr int SC_FLOATS = KBS * 4 + KBS * 8;  // 4 row-block and 8 col-block scales per block
-constexpr int NUM_EPI_WARPS = 8;
+constexpr int GRP = 2;              // contraction blocks per accumulator group (one commit)
+constexpr int STAGES = 6;
+constexpr int SC_FLOATS = 32;       // [row block r][kk] at r*4+kk, then [col block j][kk] at 16+j*4+kk
+constexpr int NUM_EPI_WARPS = 16;
 constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
 constexpr int A_STAGE = BM * KBS * KB;  // 16 KB
-constexpr int B_STAGE = BN * KBS * KB;  // 32 KB
-constexpr uint32_t TMEM_COLS = 512;     // two 256-column int32 accumulators
+constexpr int B_STAGE = BN * KBS * KB;  // 16 KB
+constexpr uint32_t TMEM_COLS = 2 * GRP * BN;   // two groups of two 128-column accumulators = 512
 
 constexpr int SMEM_A = 0;
 constexpr int SMEM_B = SMEM_A + STAGES * A_STAGE;
 constexpr int SMEM_SC = SMEM_B + STAGES * B_STAGE;
-constexpr int SMEM_BAR = SMEM_SC + SC_SLOTS * SC_FLOATS * 4;
-constexpr int NUM_BARS = 2 * STAGES + 4 + 2 * SC_SLOTS + 1;
+constexpr int SMEM_BAR = SMEM_SC + STAGES * SC_FLOATS * 4;
+constexpr int NUM_BARS = 2 * STAGES + 4 + 1;
 constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
 constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;  // + slack to align the base to 1024
 
@@ -98,29 +104,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_co
   uint8_t* sA = smem + SMEM_A;
   uint8_t* sB = smem + SMEM_B;
   float* sSc = reinterpret_cast<float*>(smem + SMEM_SC);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SMEM_BAR);
-  uint64_t* empty = full + STAGES;
-  uint64_t* tfull = empty + STAGES;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* scfull = tempty + 2;
-  uint64_t* scempty = scfull + SC_SLOTS;
-  uint64_t* drain = scempty + SC_SLOTS;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SMEM_BAR);  // per stage: A, B and scales landed
+  uint64_t* empty = full + STAGES;      // per stage: the epilogue is done with the stage
+  uint64_t* tfull = empty + STAGES;     // per accumulator group: its MMAs completed
+  uint64_t* tempty = tfull + 2;         // per accumulator group: every epilogue warp has read it
+  uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SMEM_MISC);
   volatile uint32_t* abort_flag = tmem_holder + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&full[s], 1 + 32);      // the TMA byte count plus one cp.async arrival per lane
+      mbar_init(&empty[s], NUM_EPI_WARPS);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], NUM_EPI_WARPS);
-    }
-    for (int s = 0; s < SC_SLOTS; ++s) {
-      mbar_init(&scfull[s], 32);
-      mbar_init(&scempty[s], NUM_EPI_WARPS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0u;
@@ -139,101 +139,82 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_co
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  const int num_tiles = p.tiles_m * p.tiles_n;
   const int num_kstages = (p.kblocks + KBS - 1) / KBS;
+  const int num_tiles = p.tiles_m * p.tiles_n;
+  const int my_tiles = blockIdx.x < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const int total_stages = my_tiles * num_kstages;   // this CTA's stages, in order
 
   if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    int stage = 0, sslot = 0;
-    uint32_t ph = 0, sph = 0;
-    uint32_t pending = 0, pend_ph = 0;  // stages armed by this thread, and the parity armed
-    bool ok = true;
-    for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+    // ------------------------------------------------------------------ producer warp
+    // Stage g goes to slot g % STAGES once the epilogue has finished the stage that held it (which
+    // also means the MMAs that read it have completed). Lane 0 loads A and B by TMA; every lane
+    // copies one of the stage's 32 scales (cp.async); the slot's full barrier counts both.
+    uint32_t pending = 0, pend_ph = 0;  // slots armed by lane 0, and the parity armed
+    for (int g = 0; g < total_stages; ++g) {
+      const int t = blockIdx.x + (g / num_kstages) * gridDim.x;
+      const int ks = g % num_kstages;
       const int row0 = (t % p.tiles_m) * BM, col0 = (t / p.tiles_m) * BN;
-      for (int ks = 0; ks < num_kstages; ++ks) {
-        const int kb0 = ks * KBS;
-        const int nk = min(KBS, p.kblocks - kb0);
-        if (lane == 0) {
-          if (!mbar_wait(&empty[stage], ph ^ 1u, abort_flag, p.status)) {
-            ok = false;
-          } else {
-            mbar_arrive_expect_tx(&full[stage], A_STAGE + B_STAGE);
-            pending |= 1u << stage;
-            pend_ph = (pend_ph & ~(1u << stage)) | (ph << stage);
-            uint8_t* a_dst = sA + stage * A_STAGE;
-            uint8_t* b_dst = sB + stage * B_STAGE;
-            const int k0 = kb0 * KB;
-            if (!A_MN) tma_load_2d(a_dst, &p.tma_a, &full[stage], k0, row0);
-            else tma_load_2d(a_dst, &p.tma_a, &full[stage], row0, k0);
-            if (!B_MN) {
-              tma_load_2d(b_dst, &p.tma_b, &full[stage], k0, col0);
-            } else {
-              tma_load_2d(b_dst, &p.tma_b, &full[stage], col0, k0);
-              tma_load_2d(b_dst + B_STAGE / 2, &p.tma_b, &full[stage], col0 + 128, k0);
-            }
-          }
-        }
-        ok = __shfl_sync(0xffffffffu, int(ok), 0) != 0;
-        if (!ok) break;
-        // scales of this stage: slot[kk*4 + r] = sA(row block r, kb0+kk), slot[16 + kk*8 + j] = sB(col block j)
-        ok = mbar_wait(&scempty[sslot], sph ^ 1u, abort_flag, p.status);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        float* slot = sSc + sslot * SC_FLOATS;
-        if (lane < 16) {
-          const int kk = lane >> 2, r = lane & 3;
-          const int rb = (row0 >> 5) + r;
-          if (kk < nk && rb < (p.rows >> 5))
-            cp_async_4(slot + kk * 4 + r, p.a_s + rb * p.a_s_blk + int64_t(kb0 + kk) * p.a_s_k);
-        }
-        {
-          const int kk = lane >> 3, j = lane & 7;
-          const int cb = (col0 >> 5) + j;
-          if (kk < nk && cb < (p.cols >> 5))
-            cp_async_4(slot + 16 + kk * 8 + j, p.b_s + cb * p.b_s_blk + int64_t(kb0 + kk) * p.b_s_k);
-        }
-        cp_async_mbar_arrive_noinc(&scfull[sslot]);
-        if (++stage == STAGES) { stage = 0; ph ^= 1u; }
-        if (++sslot == SC_SLOTS) { sslot = 0; sph ^= 1u; }
+      const int kb0 = ks * KBS;
+      const int nk = min(KBS, p.kblocks - kb0);
+      const int st = g % STAGES;
+      const uint32_t ph = uint32_t(g / STAGES) & 1u;
+      if (!__all_sync(0xffffffffu, mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status))) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&full[st], A_STAGE + B_STAGE);
+        pending |= 1u << st;
+        pend_ph = (pend_ph & ~(1u << st)) | (ph << st);
+        const int k0 = kb0 * KB;
+        if (!A_MN) tma_load_2d(sA + st * A_STAGE, &p.tma_a, &full[st], k0, row0);
+        else tma_load_2d(sA + st * A_STAGE, &p.tma_a, &full[st], row0, k0);
+        if (!B_MN) tma_load_2d(sB + st * B_STAGE, &p.tma_b, &full[st], k0, col0);
+        else tma_load_2d(sB + st * B_STAGE, &p.tma_b, &full[st], col0, k0);
       }
+      // lane l < 16: A scale of row block l/4, block kk = l%4; lane l >= 16: B scale of col block (l-16)/4
+      const int kk = lane & 3, blk = (lane >> 2) & 3;
+      const bool is_a = lane < 16;
+      const int gb = is_a ? (row0 >> 5) + blk : (col0 >> 5) + blk;
+      const int nb = is_a ? (p.rows >> 5) : (p.cols >> 5);
+      if (kk < nk && gb < nb) {
+        const float* src = is_a ? p.a_s + gb * p.a_s_blk + int64_t(kb0 + kk) * p.a_s_k
+                                : p.b_s + gb * p.b_s_blk + int64_t(kb0 + kk) * p.b_s_k;
+        cp_async_4(sSc + st * SC_FLOATS + lane, src);
+      }
+      cp_async_mbar_arrive_noinc(&full[st]);
     }
-    // Teardown: every TMA this thread issued must have landed before the CTA exits.
+    // Teardown: every copy issued has landed before the CTA exits.
+    asm volatile("cp.async.wait_all;" ::: "memory");
     if (lane == 0) {
       for (int s = 0; s < STAGES; ++s)
         if (pending & (1u << s)) mbar_wait_teardown(&full[s], (pend_ph >> s) & 1u, p.status);
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------------ MMA warp
     if (lane == 0) {
       constexpr uint32_t idesc = instr_desc<A_MN, B_MN>();
-      int stage = 0;
-      uint32_t ph = 0, acc = 0;
-      bool ok = true;
+      uint32_t ngroups = 0;             // accumulator groups issued so far
       bool issued = false;
-      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
-        for (int ks = 0; ok && ks < num_kstages; ++ks) {
-          const int nk = min(KBS, p.kblocks - ks * KBS);
-          if (!mbar_wait(&full[stage], ph, abort_flag, p.status)) { ok = false; break; }
+      bool ok = true;
+      for (int g = 0; ok && g < total_stages; ++g) {
+        const int st = g % STAGES;
+        const int nk = min(KBS, p.kblocks - (g % num_kstages) * KBS);
+        if (!mbar_wait(&full[st], uint32_t(g / STAGES) & 1u, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(sA + st * A_STAGE);
+        const uint32_t b_addr = smem_u32(sB + st * B_STAGE);
+        for (int k0 = 0; k0 < nk; k0 += GRP, ++ngroups) {
+          const uint32_t grp = ngroups & 1u, gph = (ngroups >> 1) & 1u;
+          if (!mbar_wait(&tempty[grp], gph ^ 1u, abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sA + stage * A_STAGE);
-          const uint32_t b_addr = smem_u32(sB + stage * B_STAGE);
-          for (int kk = 0; kk < nk; ++kk) {
-            const uint32_t buf = acc & 1u, bph = (acc >> 1) & 1u;
-            if (!mbar_wait(&tempty[buf], bph ^ 1u, abort_flag, p.status)) { ok = false; break; }
-            tc_fence_after();
+          for (int kk = k0; kk < min(nk, k0 + GRP); ++kk) {
             // K-major: the 32-byte K step moves inside the 128-byte swizzle row;
             // MN-major: it moves by 32 rows of 128 bytes (four 8-row swizzle atoms).
             const uint64_t ad = smem_desc(a_addr + (A_MN ? kk * 4096 : kk * 32), A_MN ? 16384 : 16, 1024);
             const uint64_t bd = smem_desc(b_addr + (B_MN ? kk * 4096 : kk * 32), B_MN ? 16384 : 16, 1024);
-            mma_i8(tmem_base + buf * BN, ad, bd, idesc, 0u);
-            tc_commit(&tfull[buf]);
-            issued = true;
-            ++acc;
+            mma_i8(tmem_base + (grp * GRP + uint32_t(kk - k0)) * BN, ad, bd, idesc, 0u);
           }
-          if (!ok) break;
-          tc_commit(&empty[stage]);
-          if (++stage == STAGES) { stage = 0; ph ^= 1u; }
+          tc_commit(&tfull[grp]);
+          issued = true;
         }
       }
       // Teardown: no MMA may still be writing TMEM when it is freed.
@@ -245,85 +226,92 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_co
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ epilogue warps
-    const int e = warp - 2;
-    const int sub = warp & 3;   // TMEM sub-partition this warp may access = row block in the tile
-    const int half = e >> 2;    // column half of the tile
-    const uint32_t t_lane = uint32_t(sub * 32) << 16;
-    uint32_t acc_cnt = 0;
-    int sslot = 0;
-    uint32_t sph = 0;
+    const int sub = warp & 3;           // TMEM sub-partition this warp may access = row block in the tile
+    const int cblk = (warp - 2) >> 2;   // column block of the tile
+    const uint32_t t_base = tmem_base + (uint32_t(sub * 32) << 16) + uint32_t(cblk * 32);
+    uint32_t ngroups = 0;               // accumulator groups consumed so far
     bool ok = true;
-    for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
-      const int row0 = (t % p.tiles_m) * BM, col0 = (t / p.tiles_m) * BN;
-      float acc[128];
-#pragma unroll
-      for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
-      for (int ks = 0; ks < num_kstages; ++ks) {
-        const int nk = min(KBS, p.kblocks - ks * KBS);
-        ok = __all_sync(0xffffffffu, mbar_wait(&scfull[sslot], sph, abort_flag, p.status));
-        if (!ok) break;
-        const float* slot = sSc + sslot * SC_FLOATS;
-        for (int kk = 0; kk < nk; ++kk) {
-          const float sa = slot[kk * 4 + sub];
-          float c[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) c[j] = sa * slot[16 + kk * 8 + half * 4 + j];  // fp32(sA * sB)
-          const uint32_t buf = acc_cnt & 1u, bph = (acc_cnt >> 1) & 1u;
-          ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], bph, abort_flag, p.status));
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t taddr = tmem_base + t_lane + buf * BN + half * 128;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(taddr + j * 32, r);
-            tc_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              acc[j * 32 + i] = fmaf(c[j], __int2float_rn(int(r[i])), acc[j * 32 + i]);
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[buf]);
-          ++acc_cnt;
-        }
-        if (!ok) break;
+    // Accumulate c * P from accumulator `buf`; `release` hands group `grp` back once its last
+    // accumulator is in registers.
+    auto kblock = [&](const uint32_t buf, const float c, float (&acc)[32], const bool release, const uint32_t grp) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(t_base + buf * BN, r);
+      tc_wait_ld();
+      if (release) {
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&scempty[sslot]);
-        if (++sslot == SC_SLOTS) { sslot = 0; sph ^= 1u; }
+        if (lane == 0) mbar_arrive(&tempty[grp]);
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) acc[i] = fmaf(c, __int2float_rn(int(r[i])), acc[i]);
+    };
+    // Wait until accumulator group `grp` (phase gph) holds the next contraction blocks.
+    auto wait_group = [&](const uint32_t grp, const uint32_t gph) -> bool {
+      const bool good = mbar_try_wait(&tfull[grp], gph) || mbar_wait(&tfull[grp], gph, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, good)) return false;
+      tc_fence_after();
+      return true;
+    };
+    for (int g0 = 0; ok && g0 < total_stages; g0 += num_kstages) {
+      const int t = blockIdx.x + (g0 / num_kstages) * gridDim.x;
+      const int row0 = (t % p.tiles_m) * BM, col0 = (t / p.tiles_m) * BN;
+      float acc[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
+      for (int ks = 0; ok && ks < num_kstages; ++ks) {
+        const int g = g0 + ks;
+        const int st = g % STAGES;
+        const int nk = min(KBS, p.kblocks - ks * KBS);
+        const uint32_t sph = uint32_t(g / STAGES) & 1u;
+        ok = mbar_try_wait(&full[st], sph) || mbar_wait(&full[st], sph, abort_flag, p.status);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        const float* slot = sSc + st * SC_FLOATS;
+        const float4 sa = *reinterpret_cast<const float4*>(slot + sub * 4);
+        const float4 sb = *reinterpret_cast<const float4*>(slot + 16 + cblk * 4);
+        const float c0 = sa.x * sb.x, c1 = sa.y * sb.y, c2 = sa.z * sb.z, c3 = sa.w * sb.w;  // fp32(sA * sB)
+        {  // blocks 0 and 1 of the stage
+          const uint32_t grp = ngroups & 1u;
+          if (!(ok = wait_group(grp, (ngroups >> 1) & 1u))) break;
+          kblock(grp * GRP + 0, c0, acc, nk == 1, grp);
+          if (nk >= 2) kblock(grp * GRP + 1, c1, acc, true, grp);
+          ++ngroups;
+        }
+        if (nk > GRP) {  // blocks 2 and 3
+          const uint32_t grp = ngroups & 1u;
+          if (!(ok = wait_group(grp, (ngroups >> 1) & 1u))) break;
+          kblock(grp * GRP + 0, c2, acc, nk == 3, grp);
+          if (nk == 4) kblock(grp * GRP + 1, c3, acc, true, grp);
+          ++ngroups;
+        }
+        // every accumulator of the stage has been read: its MMAs completed, the slot may be refilled
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
       }
       if (!ok) break;
-      // ---- on-chip re-quantization of the finished tile, one 32x32 block per (warp, j)
-      const int rb = (row0 >> 5) + sub;
-      if (rb < (p.rows >> 5)) {
-        const int64_t row = int64_t(rb) * 32 + lane;
-        const int ncb = p.cols >> 5;
+
+      // ---- on-chip re-quantization of this warp's 32x32 block
+      const int rbk = (row0 >> 5) + sub, cbk = (col0 >> 5) + cblk;
+      if (rbk < (p.rows >> 5) && cbk < (p.cols >> 5)) {
+        const int64_t off = (int64_t(rbk) * 32 + lane) * p.ld_y + int64_t(cbk) * 32;
+        if (p.y_q != nullptr) {
+          float m = 0.0f;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int cb = (col0 >> 5) + half * 4 + j;
-          if (cb < ncb) {
-            const float* v = acc + j * 32;
-            if (p.y_q != nullptr) {
-              float m = 0.0f;
+          for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(acc[i]));
+          const BlockQuant bq = block_quant(warp_max_nonneg(m));
+          uint32_t w[8];
 #pragma unroll
-              for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(v[i]));
-              const BlockQuant bq = block_quant(warp_max_nonneg(m));
-              uint32_t w[8];
+          for (int i = 0; i < 8; ++i)
+            w[i] = pack4(quant_byte(acc[4 * i], bq), quant_byte(acc[4 * i + 1], bq), quant_byte(acc[4 * i + 2], bq),
+                         quant_byte(acc[4 * i + 3], bq));
+          uint4* dst = reinterpret_cast<uint4*>(p.y_q + off);
+          dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+          if (lane == 0) p.y_s[int64_t(rbk) * (p.cols >> 5) + cbk] = bq.s;
+        }
+        if (p.y_f32 != nullptr) {
+          float4* dst = reinterpret_cast<float4*>(p.y_f32 + off);
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
-                w[i] = pack4(quant_byte(v[4 * i], bq), quant_byte(v[4 * i + 1], bq), quant_byte(v[4 * i + 2], bq),
-                             quant_byte(v[4 * i + 3], bq));
-              uint4* dst = reinterpret_cast<uint4*>(p.y_q + row * p.ld_y + int64_t(cb) * 32);
-              dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-              dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-              if (lane == 0) p.y_s[int64_t(rb) * ncb + cb] = bq.s;
-            }
-            if (p.y_f32 != nullptr) {
-              float4* dst = reinterpret_cast<float4*>(p.y_f32 + row * p.ld_y + int64_t(cb) * 32);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-            }
-          }
+          for (int i = 0; i < 8; ++i) dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
         }
       }
     }

@@ -31,6 +31,15 @@ __device__ __forceinline__ BlockQuant block_quant(float amax) {
   return b;
 }
 
+// Exact path of quant_byte: the IEEE quotient, clamped, rounded half to even (kept out of line so
+// that the unrolled callers stay small; it runs only for values next to a rounding tie or for
+// blocks with a subnormal scale).
+static __device__ __noinline__ uint32_t quant_byte_exact(float x, float s) {
+  float t = __fdiv_rn(x, s);
+  t = fminf(fmaxf(t, -kQMax), kQMax);
+  return __float_as_uint(t + kRoundMagic);
+}
+
 // The low byte of the result is the INT8 code of x in a block quantized with b.
 //
 // Fast path (s normal): t = RN(x * RN(1/s)). With e = x/s exact and |e| <= 127 (1 + 2^-23),
@@ -46,9 +55,7 @@ __device__ __forceinline__ uint32_t quant_byte(float x, const BlockQuant& b) {
   } else if (b.mode == 0) {
     return 0u;
   }
-  float t = __fdiv_rn(x, b.s);
-  t = fminf(fmaxf(t, -kQMax), kQMax);
-  return __float_as_uint(t + kRoundMagic);
+  return quant_byte_exact(x, b.s);
 }
 
 // Pack the low bytes of four words into one word (a in byte 0 ... d in byte 3).
