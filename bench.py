@@ -48,6 +48,10 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     p.add_argument("--cpu-sample-tokens", type=int, default=1024)
+    p.add_argument("--sweep", action="store_true",
+                   help="time the memory-bound kernels on the M x 4096 sweep instead of the step")
+    p.add_argument("--sweep-m", type=int, nargs="*", default=[1024, 8192, 65536])
+    p.add_argument("--sweep-ops", nargs="*", default=["quantize_bf16", "dequantize_bf16", "gelu_i8", "layernorm_i8"])
     return p.parse_args()
 
 
@@ -445,8 +449,62 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_sweep(args):
+    """Memory-bound sweep: quantize (bf16 in), dequantize (bf16 out), GELU_i8 and LayerNorm_i8 on
+    M x 4096 tensors, M in {1024, 8192, 65536}; N(0,1) with 1% of the channels x100. One JSON line
+    with GB/s (algorithmic bytes: read once, write once) and the fraction of the measured HBM copy
+    bandwidth per kernel and size."""
+    import torch
+    import int8_fully_quantized_b200 as jf
+    from inputs import synthetic as S
+    torch.cuda.set_device(0)
+    jf.load_library()
+    peaks, peak_src = load_peaks()
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    H = 4096
+    out = {}
+    for M in args.sweep_m:
+        x = S.to_bf16_bits(S.memory_sweep_input(0, M, H))
+        xb = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+        del x
+        Q = jf.quantize_block(xb)
+        Y = jf.empty_qtensor(M, H)
+        yb = torch.empty((M, H), dtype=torch.bfloat16, device="cuda")
+        gamma = torch.ones(H, device="cuda")
+        beta = torch.zeros(H, device="cuda")
+        ops = {
+            "quantize_bf16": (lambda: jf.jf_quantize_block(xb, Y.q, Y.s), bytes_quant(M, H, 2)),
+            "dequantize_bf16": (lambda: jf.jf_dequantize_block(Q.q, Q.s, yb), M * H * 3 + (M // 32) * (H // 32) * 4),
+            "gelu_i8": (lambda: jf.jf_gelu_i8(Q, Y), bytes_i8_op(M, H)),
+            "layernorm_i8": (lambda: jf.jf_layernorm_i8(Q, gamma, beta, 1e-5, Y), bytes_i8_op(M, H, 8 * H)),
+        }
+        for name, (fn, nbytes) in ops.items():
+            if name not in args.sweep_ops:
+                continue
+            for _ in range(3):
+                flush.zero_()
+                fn()
+            ts = []
+            for _ in range(max(5, args.steps // 5)):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(); fn(); b.record()
+                ts.append((a, b))
+            torch.cuda.synchronize()
+            ms = statistics.median(a.elapsed_time(b) for a, b in ts)
+            gbs = nbytes / (ms * 1e-3) / 1e9
+            out[f"{name}@M={M}"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+        del xb, Q, Y, yb
+    assert jf.jf_device_status() == 0
+    print(json.dumps({"sweep": out, "hbm_peak_gbs": peaks["hbm_gbs"], "peak_source": peak_src,
+                      "l2": "flushed before every timed launch"}), flush=True)
+
+
 def main():
     args = parse_args()
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -78,15 +78,6 @@ struct Vec<__half> {
   }
 };
 
-// Codes of `n` (4 or 8) values -> 4 or 8 bytes.
-template <int N>
-__device__ __forceinline__ void quant_pack(const float* v, const BlockQuant& b, uint32_t* out) {
-#pragma unroll
-  for (int i = 0; i < N / 4; ++i)
-    out[i] = pack4(quant_byte(v[4 * i], b), quant_byte(v[4 * i + 1], b), quant_byte(v[4 * i + 2], b),
-                   quant_byte(v[4 * i + 3], b));
-}
-
 // ---------------------------------------------------------------------------------------------
 // a1: quantize. One warp per 32x32 block. A block row of T is VPR 16-byte vectors; lane l reads
 // vector column l % VPR of rows l / VPR + t * (32 / VPR), so each load instruction covers whole
@@ -94,36 +85,51 @@ __device__ __forceinline__ void quant_pack(const float* v, const BlockQuant& b, 
 // ---------------------------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(256, 4) quantize_kernel(const T* __restrict__ x, int64_t R, int64_t C,
-                                                       int8_t* __restrict__ q, float* __restrict__ s) {
+                                                          int8_t* __restrict__ q, float* __restrict__ s) {
   constexpr int EPV = Vec<T>::kElems;      // elements per 16-byte vector
-  constexpr int VPR = 32 / EPV;            // vectors per block row
+  constexpr int VPR = 32 / EPV;            // vectors per block row (= vectors per lane)
   constexpr int RSTEP = 32 / VPR;          // rows between a lane's vectors
   const int lane = threadIdx.x & 31;
   const int64_t nbc = C >> 5;
   const int64_t nblocks = (R >> 5) * nbc;
   const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
   const int r0 = lane / VPR, vc = lane % VPR;
-  for (int64_t b = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; b < nblocks; b += nwarps) {
+  auto src_of = [&](int64_t b) {
     const int64_t bi = b / nbc, bj = b - bi * nbc;
-    const T* src = x + (bi * 32 + r0) * C + bj * 32 + vc * EPV;
-    float v[VPR][EPV];
+    return x + (bi * 32 + r0) * C + bj * 32 + vc * EPV;
+  };
+  int64_t b = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  uint4 raw[VPR];
+  if (b < nblocks) {
+    const T* src = src_of(b);
 #pragma unroll
-    for (int t = 0; t < VPR; ++t) Vec<T>::unpack(ld_stream_v4(src + int64_t(t) * RSTEP * C), v[t]);
+    for (int t = 0; t < VPR; ++t) raw[t] = ld_stream_v4(src + int64_t(t) * RSTEP * C);
+  }
+  for (; b < nblocks; b += nwarps) {
+    float v[VPR * EPV];
+#pragma unroll
+    for (int t = 0; t < VPR; ++t) Vec<T>::unpack(raw[t], *reinterpret_cast<float(*)[EPV]>(v + t * EPV));
+    // the next block's loads are in flight while this block is quantized
+    const int64_t bn = b + nwarps;
+    if (bn < nblocks) {
+      const T* src = src_of(bn);
+#pragma unroll
+      for (int t = 0; t < VPR; ++t) raw[t] = ld_stream_v4(src + int64_t(t) * RSTEP * C);
+    }
     float m = 0.0f;
 #pragma unroll
-    for (int t = 0; t < VPR; ++t)
-#pragma unroll
-      for (int i = 0; i < EPV; ++i) m = fmaxf(m, fabsf(v[t][i]));
+    for (int i = 0; i < VPR * EPV; ++i) m = fmaxf(m, fabsf(v[i]));
     const BlockQuant bq = block_quant(warp_max_nonneg(m));
+    uint32_t w[VPR * EPV / 4];
+    quant_pack<VPR * EPV>(v, bq, w);
+    const int64_t bi = b / nbc, bj = b - bi * nbc;
     int8_t* dst = q + (bi * 32 + r0) * C + bj * 32 + vc * EPV;
 #pragma unroll
     for (int t = 0; t < VPR; ++t) {
-      uint32_t w[EPV / 4];
-      quant_pack<EPV>(v[t], bq, w);
       if constexpr (EPV == 4) {
-        *reinterpret_cast<uint32_t*>(dst + int64_t(t) * RSTEP * C) = w[0];
+        *reinterpret_cast<uint32_t*>(dst + int64_t(t) * RSTEP * C) = w[t];
       } else {
-        *reinterpret_cast<uint2*>(dst + int64_t(t) * RSTEP * C) = make_uint2(w[0], w[1]);
+        *reinterpret_cast<uint2*>(dst + int64_t(t) * RSTEP * C) = make_uint2(w[2 * t], w[2 * t + 1]);
       }
     }
     if (lane == 0) s[b] = bq.s;
@@ -184,10 +190,18 @@ __global__ void __launch_bounds__(256, 4) dequantize_kernel(const int8_t* __rest
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ float gelu_f32(float x) { return 0.5f * x * erfcf(x * -0.70710678118654752440f); }
 
-__global__ void __launch_bounds__(256, 4) gelu_i8_kernel(const int8_t* __restrict__ q, const float* __restrict__ s,
-                                                      int64_t R, int64_t C, int8_t* __restrict__ qo,
-                                                      float* __restrict__ so) {
-  const int lane = threadIdx.x & 31;
+constexpr int kGeluWarps = 8;
+
+__global__ void __launch_bounds__(32 * kGeluWarps, 4) gelu_i8_kernel(const int8_t* __restrict__ q,
+                                                                    const float* __restrict__ s, int64_t R,
+                                                                    int64_t C, int8_t* __restrict__ qo,
+                                                                    float* __restrict__ so) {
+  // A block's input has at most 255 distinct values q * s, so each warp first tabulates GELU of all
+  // of them (8 evaluations per lane instead of 32) and then looks its 32 values up; the results are
+  // the same as evaluating GELU per element.
+  __shared__ float table[kGeluWarps][256];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  float* tab = table[wib];
   const int64_t nbc = C >> 5;
   const int64_t nblocks = (R >> 5) * nbc;
   const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
@@ -198,19 +212,26 @@ __global__ void __launch_bounds__(256, 4) gelu_i8_kernel(const int8_t* __restric
     const int64_t off = (bi * 32 + r0) * C + bj * 32 + c0;
     const uint4 a0 = ld_stream_v4(q + off);
     const uint4 a1 = ld_stream_v4(q + off + 16 * C);
+    // table[u] = GELU(fp32(u - 128) * s) for u = 1..255 (code u - 128)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int u = lane + 32 * j;
+      tab[u] = gelu_f32(float(u - 128) * sc);
+    }
+    __syncwarp();
     const uint32_t w[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
     float v[32];
     float m = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      float g[4];
-      i8x4_to_f32(w[i], g);
+      const uint32_t u = w[i] ^ 0x80808080u;  // code + 128 in each byte
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        v[4 * i + j] = gelu_f32(g[j] * sc);
+        v[4 * i + j] = tab[(u >> (8 * j)) & 0xFFu];
         m = fmaxf(m, fabsf(v[4 * i + j]));
       }
     }
+    __syncwarp();  // the table is rewritten for the next block only after every lane has read it
     const BlockQuant bq = block_quant(warp_max_nonneg(m));
     uint32_t o[8];
     quant_pack<32>(v, bq, o);
@@ -246,9 +267,25 @@ __global__ void __launch_bounds__(kLnThreads) layernorm_i8_kernel(const int8_t* 
   {
     const int8_t* row = qs + int64_t(warp) * H;
     double sum = 0.0, sq = 0.0;
-    for (int64_t ch = lane; ch < (H >> 4); ch += 32) {
-      const uint4 a = ld_stream_v4(row + ch * 16);
-      const float sc = __ldg(ss + (ch >> 1));
+    constexpr int kUnroll = 8;  // 16-byte chunks of the row a lane keeps in flight
+    for (int64_t ch0 = lane; ch0 < (H >> 4); ch0 += 32 * kUnroll) {
+      uint4 av[kUnroll];
+      float scv[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t ch = ch0 + 32 * u;
+        if (ch < (H >> 4)) {
+          av[u] = ld_stream_v4(row + ch * 16);
+          scv[u] = __ldg(ss + (ch >> 1));
+        } else {
+          av[u] = make_uint4(0u, 0u, 0u, 0u);
+          scv[u] = 0.0f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+      const uint4 a = av[u];
+      const float sc = scv[u];
       const uint32_t w[4] = {a.x, a.y, a.z, a.w};
       float ps = 0.0f, pq = 0.0f;
 #pragma unroll
@@ -264,6 +301,7 @@ __global__ void __launch_bounds__(kLnThreads) layernorm_i8_kernel(const int8_t* 
       }
       sum += double(ps);
       sq += double(pq);
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -361,7 +399,7 @@ cudaError_t launch_dequantize(const int8_t* q, const float* s, int64_t R, int64_
 cudaError_t launch_gelu_i8(const int8_t* q, const float* s, int64_t R, int64_t C, int8_t* qo, float* so,
                            int sm_count, cudaStream_t st) {
   const int grid = grid_for_blocks((R / 32) * (C / 32), sm_count);
-  gelu_i8_kernel<<<grid, 256, 0, st>>>(q, s, R, C, qo, so);
+  gelu_i8_kernel<<<grid, 32 * kGeluWarps, 0, st>>>(q, s, R, C, qo, so);
   return cudaGetLastError();
 }
 

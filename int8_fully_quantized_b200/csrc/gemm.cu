@@ -299,10 +299,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_co
           for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(acc[i]));
           const BlockQuant bq = block_quant(warp_max_nonneg(m));
           uint32_t w[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            w[i] = pack4(quant_byte(acc[4 * i], bq), quant_byte(acc[4 * i + 1], bq), quant_byte(acc[4 * i + 2], bq),
-                         quant_byte(acc[4 * i + 3], bq));
+          quant_pack<32>(acc, bq, w);
           uint4* dst = reinterpret_cast<uint4*>(p.y_q + off);
           dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
           dst[1] = make_uint4(w[4], w[5], w[6], w[7]);

@@ -58,6 +58,40 @@ __device__ __forceinline__ uint32_t quant_byte(float x, const BlockQuant& b) {
   return quant_byte_exact(x, b.s);
 }
 
+// Codes of N values (N a multiple of 8), packed four to a word (value 4i in byte 0 of word i).
+// The fast path of quant_byte runs branch-free on groups of 8 values; one test per group looks for a
+// value next to a rounding tie (rare), and only then is the group recomputed exactly.
+template <int N>
+__device__ __forceinline__ void quant_pack(const float* v, const BlockQuant& b, uint32_t* out) {
+  static_assert(N % 8 == 0, "values are handled in groups of eight");
+#pragma unroll
+  for (int g = 0; g < N; g += 8) {
+    uint32_t c[8];
+    if (b.mode == 2) {
+      bool near_tie = false;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float t = v[g + i] * b.inv;
+        const float tp = t + kRoundMagic;
+        near_tie |= !(fabsf(t - (tp - kRoundMagic)) < 0.49993896484375f);  // 0.5 - 2^-14
+        c[i] = __float_as_uint(tp);
+      }
+      if (near_tie) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) c[i] = quant_byte(v[g + i], b);
+      }
+    } else if (b.mode == 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) c[i] = 0u;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) c[i] = quant_byte_exact(v[g + i], b.s);
+    }
+    out[g / 4] = __byte_perm(__byte_perm(c[0], c[1], 0x0040), __byte_perm(c[2], c[3], 0x0040), 0x5410);
+    out[g / 4 + 1] = __byte_perm(__byte_perm(c[4], c[5], 0x0040), __byte_perm(c[6], c[7], 0x0040), 0x5410);
+  }
+}
+
 // Pack the low bytes of four words into one word (a in byte 0 ... d in byte 3).
 __device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
