@@ -318,12 +318,15 @@ def run_ours(args):
 
 
 def _load_traffic(kernel_op):
-    """dram read + write bytes per launch of the dominant kernel from the committed ncu summary
-    (profiles/gemm_traffic.json), or None when no capture of the current kernel exists."""
+    """DRAM read + write bytes per launch of the dominant kernel from the committed ncu capture
+    (profiles/gemm_traffic.json), or None when that capture was taken of other kernel sources."""
     path = os.path.join(ROOT, "profiles", "gemm_traffic.json")
     try:
+        from int8_fully_quantized_b200 import build_lib
         with open(path) as f:
             d = json.load(f)
+        if d.get("source_hash") != build_lib.source_hash():
+            return None
         v = d.get(kernel_op)
         return None if v is None else int(v)
     except Exception:

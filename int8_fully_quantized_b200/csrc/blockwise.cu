@@ -242,17 +242,18 @@ __global__ void __launch_bounds__(32 * kGeluWarps, 4) gelu_i8_kernel(const int8_
 }
 
 // ---------------------------------------------------------------------------------------------
-// a7: LayerNorm_i8. One CTA of 32 warps per 32-row strip [32, H].
-//   phase 1: warp w reduces row w: sum and sum of squares of x = fp32(q) * s (chunk partials of
-//            16 values in fp32, accumulated in fp64), then mean, biased variance and
+// a7: LayerNorm_i8. One CTA of 16 warps per 32-row strip [32, H]; two CTAs share an SM so that
+// one's reduction overlaps the other's output phase.
+//   phase 1: warp w reduces rows w and w + 16: sum and sum of squares of x = fp32(q) * s (chunk
+//            partials of 16 values in fp32, accumulated in fp64), then mean, biased variance and
 //            rstd = 1 / sqrt(var + eps) in fp64, kept in shared memory.
-//   phase 2: warp w handles column blocks w, w + 32, ...: y = (x - mean) * rstd * gamma + beta in
+//   phase 2: warp w handles column blocks w, w + 16, ...: y = (x - mean) * rstd * gamma + beta in
 //            fp32, block absmax, per-block re-quantization. The strip is read a second time; it
 //            is at most 32 * H bytes and is still in L2.
 // ---------------------------------------------------------------------------------------------
-constexpr int kLnThreads = 1024;
+constexpr int kLnThreads = 512;
 
-__global__ void __launch_bounds__(kLnThreads) layernorm_i8_kernel(const int8_t* __restrict__ q,
+__global__ void __launch_bounds__(kLnThreads, 2) layernorm_i8_kernel(const int8_t* __restrict__ q,
                                                                   const float* __restrict__ s, int64_t R,
                                                                   int64_t H, const float* __restrict__ gamma,
                                                                   const float* __restrict__ beta, float eps,
@@ -264,8 +265,8 @@ __global__ void __launch_bounds__(kLnThreads) layernorm_i8_kernel(const int8_t* 
   const int64_t nbc = H >> 5;
   const int8_t* qs = q + strip * 32 * H;
   const float* ss = s + strip * nbc;
-  {
-    const int8_t* row = qs + int64_t(warp) * H;
+  for (int rw = warp; rw < 32; rw += kLnThreads / 32) {
+    const int8_t* row = qs + int64_t(rw) * H;
     double sum = 0.0, sq = 0.0;
     constexpr int kUnroll = 8;  // 16-byte chunks of the row a lane keeps in flight
     for (int64_t ch0 = lane; ch0 < (H >> 4); ch0 += 32 * kUnroll) {
@@ -312,8 +313,8 @@ __global__ void __launch_bounds__(kLnThreads) layernorm_i8_kernel(const int8_t* 
       const double mean = sum / double(H);
       double var = sq / double(H) - mean * mean;
       var = var > 0.0 ? var : 0.0;
-      s_mean[warp] = float(mean);
-      s_rstd[warp] = float(1.0 / sqrt(var + double(eps)));
+      s_mean[rw] = float(mean);
+      s_rstd[rw] = float(1.0 / sqrt(var + double(eps)));
     }
   }
   __syncthreads();
