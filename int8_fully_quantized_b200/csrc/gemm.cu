@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_co
     auto kblock = [&](const uint32_t buf, const float c, float (&acc)[32], const bool release, const uint32_t grp) {
       uint32_t r[32];
       tmem_ld_32x32b_x32(t_base + buf * BN, r);
-      tc_wait_ld();
+      tc_wait_ld(r);
       if (release) {
         tc_fence_before();
         __syncwarp();
