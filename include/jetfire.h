@@ -109,6 +109,21 @@ JF_API int jf_dequantize_block(const int8_t* q, const float* s, int64_t rows, in
 JF_API int jf_linear_fwd(jf_cqtensor X, jf_cqtensor W, jf_qtensor Y, float* y_f32, void* stream);
 
 /*
+ * f1. Linear forward with GELU fused into the re-quantization epilogue (summary, "Approach":
+ *     quantization happens on-chip; here the activation that follows fc1 happens there too).
+ *   X [M, K], W [N, K] as in jf_linear_fwd. With P the fp32 pre-activation that jf_linear_fwd
+ *   computes, Y = requant(GELU(P)) per 32x32 block, GELU in its exact erf form applied to the fp32
+ *   P (not to its INT8 re-quantization), so the result differs from jf_linear_fwd followed by
+ *   jf_gelu_i8 by that one rounding step.
+ *   Y     [M, N] output; Y.q and Y.s are required.
+ *   Ypre  optional [M, N] output: requant(P), identical to jf_linear_fwd's Y. Pass Ypre.q = NULL to
+ *         skip it; it is what the backward of GELU needs.
+ *   Errors as jf_linear_fwd; JF_ERR_NULL when Y.q is NULL; JF_ERR_ALIAS when any two of the
+ *   outputs, or an output and an input, overlap.
+ */
+JF_API int jf_linear_fwd_gelu(jf_cqtensor X, jf_cqtensor W, jf_qtensor Y, jf_qtensor Ypre, void* stream);
+
+/*
  * a4. Input gradient dX = dY W (the INT8 backward of the linear layer).
  *   dY [M, N], W [N, K] (read re-blocked along N, no transpose pass), dX [M, K] (output).
  *   dX(m, k) = sum_nb fp32(sdY(m/32, nb) sW(nb, k/32)) * sum_{n in nb} dYq(m, n) Wq(n, k).

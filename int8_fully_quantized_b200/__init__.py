@@ -23,8 +23,9 @@ from .build_lib import LIB_PATH
 
 __all__ = [
     "QTensor", "JetfireError", "load_library", "empty_qtensor", "jf_quantize_block", "jf_dequantize_block",
-    "jf_linear_fwd", "jf_linear_dgrad", "jf_linear_wgrad", "jf_gelu_i8", "jf_layernorm_i8", "jf_strerror",
-    "jf_device_status", "jf_sm_count", "quantize_block", "dequantize_block", "linear_fwd", "linear_dgrad",
+    "jf_linear_fwd", "jf_linear_fwd_gelu", "jf_linear_dgrad", "jf_linear_wgrad", "jf_gelu_i8", "jf_layernorm_i8",
+    "jf_strerror", "jf_device_status", "jf_sm_count", "quantize_block", "dequantize_block", "linear_fwd",
+    "linear_fwd_gelu", "linear_dgrad",
     "linear_wgrad", "gelu_i8", "layernorm_i8", "EXPORTED_SYMBOLS", "JF_F32", "JF_BF16", "JF_F16",
 ]
 
@@ -32,7 +33,8 @@ JF_F32, JF_BF16, JF_F16 = 0, 1, 2
 _DTYPES = {torch.float32: JF_F32, torch.bfloat16: JF_BF16, torch.float16: JF_F16}
 
 EXPORTED_SYMBOLS = (
-    "jf_quantize_block", "jf_dequantize_block", "jf_linear_fwd", "jf_linear_dgrad", "jf_linear_wgrad",
+    "jf_quantize_block", "jf_dequantize_block", "jf_linear_fwd", "jf_linear_fwd_gelu", "jf_linear_dgrad",
+    "jf_linear_wgrad",
     "jf_gelu_i8", "jf_layernorm_i8", "jf_strerror", "jf_device_status", "jf_sm_count",
 )
 
@@ -71,6 +73,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.jf_dequantize_block.argtypes = [vp, vp, i64, i64, vp, i32, vp]
     for name in ("jf_linear_fwd", "jf_linear_dgrad", "jf_linear_wgrad"):
         getattr(lib, name).argtypes = [_CQ, _CQ, _Q, vp, vp]
+    lib.jf_linear_fwd_gelu.argtypes = [_CQ, _CQ, _Q, _Q, vp]
     lib.jf_gelu_i8.argtypes = [_CQ, _Q, vp]
     lib.jf_layernorm_i8.argtypes = [_CQ, vp, vp, ctypes.c_float, _Q, vp]
     lib.jf_strerror.argtypes = [i32]
@@ -154,6 +157,12 @@ def jf_linear_fwd(X: QTensor, W: QTensor, Y: Optional[QTensor], y_f32: Optional[
     _check(lib.jf_linear_fwd(_cq(X), _cq(W), _q(Y, X.rows, W.rows), _ptr(y_f32), _stream(stream)), "jf_linear_fwd")
 
 
+def jf_linear_fwd_gelu(X: QTensor, W: QTensor, Y: QTensor, Ypre: Optional[QTensor] = None, stream=None) -> None:
+    lib = load_library()
+    _check(lib.jf_linear_fwd_gelu(_cq(X), _cq(W), _q(Y, X.rows, W.rows), _q(Ypre, X.rows, W.rows), _stream(stream)),
+           "jf_linear_fwd_gelu")
+
+
 def jf_linear_dgrad(dY: QTensor, W: QTensor, dX: Optional[QTensor], dx_f32: Optional[torch.Tensor] = None,
                     stream=None) -> None:
     lib = load_library()
@@ -210,6 +219,15 @@ def linear_fwd(X: QTensor, W: QTensor, want_f32: bool = False, stream=None):
     yf = torch.empty((X.rows, W.rows), dtype=torch.float32, device=X.q.device) if want_f32 else None
     jf_linear_fwd(X, W, Y, yf, stream)
     return (Y, yf) if want_f32 else Y
+
+
+def linear_fwd_gelu(X: QTensor, W: QTensor, want_pre: bool = False, stream=None):
+    """Y = requant(GELU(X W^T)) with GELU applied on chip; with ``want_pre`` also the re-quantized
+    pre-activation (the same tensor linear_fwd returns)."""
+    Y = empty_qtensor(X.rows, W.rows, X.q.device)
+    P = empty_qtensor(X.rows, W.rows, X.q.device) if want_pre else None
+    jf_linear_fwd_gelu(X, W, Y, P, stream)
+    return (Y, P) if want_pre else Y
 
 
 def linear_dgrad(dY: QTensor, W: QTensor, want_f32: bool = False, stream=None):

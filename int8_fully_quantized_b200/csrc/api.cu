@@ -84,25 +84,31 @@ int64_t qbytes(const jf_cqtensor& t) { return t.rows * t.cols; }
 int64_t sbytes(int64_t r, int64_t c) { return (r / 32) * (c / 32) * 4; }
 
 // Shared validation + launch of the three GEMMs. A/B are the stored operands.
+// `pre` (activation kActGelu only; q may be NULL) receives the re-quantized pre-activation.
 int gemm_call(int mode, const jf_cqtensor& A, const jf_cqtensor& B, const jf_qtensor& Y, float* y_f32,
-              int64_t rows, int64_t cols, int64_t depth, void* stream) {
+              int64_t rows, int64_t cols, int64_t depth, void* stream, int act = jf::kActNone,
+              jf_qtensor pre = jf_qtensor{nullptr, nullptr, 0, 0}) {
   int st;
   if ((st = check_cq(A)) != JF_OK) return st;
   if ((st = check_cq(B)) != JF_OK) return st;
   if ((st = check_q(Y, false)) != JF_OK) return st;
   if (Y.rows != rows || Y.cols != cols) return JF_ERR_SHAPE;
+  if (pre.q != nullptr) {
+    if ((st = check_q(pre, true)) != JF_OK) return st;
+    if (pre.rows != rows || pre.cols != cols) return JF_ERR_SHAPE;
+  }
   if (rows == 0 || cols == 0) return JF_OK;
   if (Y.q == nullptr && y_f32 == nullptr) return JF_ERR_NULL;
   if (y_f32 != nullptr && !aligned(y_f32, 16)) return JF_ERR_ALIGN;
   // outputs must not overlap inputs (nor each other)
   const void* ins[4] = {A.q, A.s, B.q, B.s};
   const int64_t in_n[4] = {qbytes(A), sbytes(A.rows, A.cols), qbytes(B), sbytes(B.rows, B.cols)};
-  const void* outs[3] = {Y.q, Y.q ? Y.s : nullptr, y_f32};
-  const int64_t out_n[3] = {rows * cols, sbytes(rows, cols), rows * cols * 4};
-  for (int o = 0; o < 3; ++o) {
+  const void* outs[5] = {Y.q, Y.q ? Y.s : nullptr, y_f32, pre.q, pre.q ? pre.s : nullptr};
+  const int64_t out_n[5] = {rows * cols, sbytes(rows, cols), rows * cols * 4, rows * cols, sbytes(rows, cols)};
+  for (int o = 0; o < 5; ++o) {
     for (int i = 0; i < 4; ++i)
       if (overlap(outs[o], out_n[o], ins[i], in_n[i])) return JF_ERR_ALIAS;
-    for (int o2 = o + 1; o2 < 3; ++o2)
+    for (int o2 = o + 1; o2 < 5; ++o2)
       if (overlap(outs[o], out_n[o], outs[o2], out_n[o2])) return JF_ERR_ALIAS;
   }
   const DevInfo d = device_info();
@@ -121,6 +127,9 @@ int gemm_call(int mode, const jf_cqtensor& A, const jf_cqtensor& B, const jf_qte
   g.y_q = Y.q;
   g.y_s = Y.q ? Y.s : nullptr;
   g.y_f32 = y_f32;
+  g.act = act;
+  g.pre_q = pre.q;
+  g.pre_s = pre.q ? pre.s : nullptr;
   g.status = d.status;
   if (depth == 0) {
     // empty contraction: the result is exactly zero (codes 0, scales 0)
@@ -131,6 +140,11 @@ int gemm_call(int mode, const jf_cqtensor& A, const jf_cqtensor& B, const jf_qte
       if (e == cudaSuccess) e = cudaMemsetAsync(Y.s, 0, size_t(sbytes(rows, cols)), s);
     }
     if (e == cudaSuccess && y_f32) e = cudaMemsetAsync(y_f32, 0, size_t(rows * cols * 4), s);
+    // GELU(0) = 0: the fused output and the pre-activation are zero as well
+    if (e == cudaSuccess && pre.q) {
+      e = cudaMemsetAsync(pre.q, 0, size_t(rows * cols), s);
+      if (e == cudaSuccess) e = cudaMemsetAsync(pre.s, 0, size_t(sbytes(rows, cols)), s);
+    }
     return cuda_status(e);
   }
   return cuda_status(jf::launch_gemm(g, d.sm_count, static_cast<cudaStream_t>(stream)));
@@ -174,6 +188,13 @@ int jf_linear_fwd(jf_cqtensor X, jf_cqtensor W, jf_qtensor Y, float* y_f32, void
   if (!dims_ok(X.rows, X.cols) || !dims_ok(W.rows, W.cols)) return JF_ERR_SHAPE;
   if (X.cols != W.cols) return JF_ERR_SHAPE;
   return gemm_call(jf::kFwd, X, W, Y, y_f32, X.rows, W.rows, X.cols, stream);
+}
+
+int jf_linear_fwd_gelu(jf_cqtensor X, jf_cqtensor W, jf_qtensor Y, jf_qtensor Ypre, void* stream) {
+  if (!dims_ok(X.rows, X.cols) || !dims_ok(W.rows, W.cols)) return JF_ERR_SHAPE;
+  if (X.cols != W.cols) return JF_ERR_SHAPE;
+  if (Y.q == nullptr && X.rows != 0 && W.rows != 0) return JF_ERR_NULL;
+  return gemm_call(jf::kFwd, X, W, Y, nullptr, X.rows, W.rows, X.cols, stream, jf::kActGelu, Ypre);
 }
 
 int jf_linear_dgrad(jf_cqtensor dY, jf_cqtensor W, jf_qtensor dX, float* dx_f32, void* stream) {

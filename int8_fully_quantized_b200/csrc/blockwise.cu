@@ -12,6 +12,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include "act.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
 #include "quant.cuh"
@@ -185,10 +186,8 @@ __global__ void __launch_bounds__(256, 4) dequantize_kernel(const int8_t* __rest
 // ---------------------------------------------------------------------------------------------
 // a6: GELU_i8. One warp per block; the block is 64 16-byte chunks, lane l takes chunks l and
 // l + 32, i.e. columns 16 (l % 2) .. +15 of rows l / 2 and 16 + l / 2.
-// GELU(x) = x Phi(x) = 0.5 x erfc(-x / sqrt 2): the erfc form keeps its relative accuracy for
-// negative x, where 1 + erf(x / sqrt 2) cancels.
+// GELU is evaluated by gelu_f32 (act.cuh), in its erfc form.
 // ---------------------------------------------------------------------------------------------
-__device__ __forceinline__ float gelu_f32(float x) { return 0.5f * x * erfcf(x * -0.70710678118654752440f); }
 
 constexpr int kGeluWarps = 8;
 

@@ -35,6 +35,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include "act.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
 #include "quant.cuh"
@@ -72,6 +73,9 @@ struct __align__(64) GemmParams {
   int8_t* y_q;
   float* y_s;
   float* y_f32;
+  int8_t* pre_q;
+  float* pre_s;
+  int act;
   int64_t ld_y;
   unsigned int* status;
   int rows, cols, kblocks;
@@ -95,6 +99,21 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
 __device__ __forceinline__ void mbar_wait_teardown(uint64_t* bar, uint32_t parity, unsigned int* status) {
   uint32_t dummy = 0;
   mbar_wait(bar, parity, &dummy, status);
+}
+
+// Re-quantize one warp's 32x32 fp32 block (lane = row; the row's 32 values in acc) and store its
+// codes at q (lane's row, ld_y-strided by the caller's offset) and its scale at *s.
+__device__ __forceinline__ void store_block_q(const float (&acc)[32], int8_t* q, float* s, const int lane) {
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(acc[i]));
+  const BlockQuant bq = block_quant(warp_max_nonneg(m));
+  uint32_t w[8];
+  quant_pack<32>(acc, bq, w);
+  uint4* dst = reinterpret_cast<uint4*>(q);
+  dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  if (lane == 0) *s = bq.s;
 }
 
 template <bool A_MN, bool B_MN>
@@ -293,18 +312,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_co
       const int rbk = (row0 >> 5) + sub, cbk = (col0 >> 5) + cblk;
       if (rbk < (p.rows >> 5) && cbk < (p.cols >> 5)) {
         const int64_t off = (int64_t(rbk) * 32 + lane) * p.ld_y + int64_t(cbk) * 32;
-        if (p.y_q != nullptr) {
-          float m = 0.0f;
+        const int64_t soff = int64_t(rbk) * (p.cols >> 5) + cbk;
+        if (p.act == kActGelu) {
+          // fused activation: the fp32 pre-activation is re-quantized (when asked for) and GELU is
+          // applied to it on chip, so neither ever makes an HBM round trip in fp32
+          if (p.pre_q != nullptr) store_block_q(acc, p.pre_q + off, p.pre_s + soff, lane);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(acc[i]));
-          const BlockQuant bq = block_quant(warp_max_nonneg(m));
-          uint32_t w[8];
-          quant_pack<32>(acc, bq, w);
-          uint4* dst = reinterpret_cast<uint4*>(p.y_q + off);
-          dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-          dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-          if (lane == 0) p.y_s[int64_t(rbk) * (p.cols >> 5) + cbk] = bq.s;
+          for (int i = 0; i < 32; ++i) acc[i] = gelu_f32(acc[i]);
         }
+        if (p.y_q != nullptr) store_block_q(acc, p.y_q + off, p.y_s + soff, lane);
         if (p.y_f32 != nullptr) {
           float4* dst = reinterpret_cast<float4*>(p.y_f32 + off);
 #pragma unroll
@@ -400,6 +416,9 @@ cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t st) {
   prm.y_q = g.y_q;
   prm.y_s = g.y_s;
   prm.y_f32 = g.y_f32;
+  prm.act = g.act;
+  prm.pre_q = g.pre_q;
+  prm.pre_s = g.pre_s;
   prm.ld_y = g.cols;
   prm.status = g.status;
   prm.rows = int(g.rows);

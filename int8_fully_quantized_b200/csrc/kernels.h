@@ -19,6 +19,7 @@ cudaError_t launch_layernorm_i8(const int8_t* q, const float* s, int64_t R, int6
 // fp32(sA(r/32, kb) * sB(c/32, kb)) * sum_{k in kb} A(r, k) B(c, k), re-quantized per 32x32 block.
 // The operand views differ per mode (see gemm.cu).
 enum GemmMode { kFwd = 0, kDgrad = 1, kWgrad = 2 };
+enum GemmAct { kActNone = 0, kActGelu = 1 };
 
 struct GemmArgs {
   int mode;
@@ -31,6 +32,9 @@ struct GemmArgs {
   int8_t* y_q;                // nullable
   float* y_s;                 // non-null when y_q is
   float* y_f32;               // nullable
+  int act;                    // GemmAct: activation applied to the fp32 result before y is written
+  int8_t* pre_q;              // nullable (kActGelu only): the re-quantized pre-activation
+  float* pre_s;               // non-null when pre_q is
   unsigned int* status;       // device status word (bit flags of ptx.cuh)
 };
 

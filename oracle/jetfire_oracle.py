@@ -42,7 +42,7 @@ QMAX = 127
 
 __all__ = [
     "BLOCK", "QMAX", "bf16_bits_to_f32", "f32_to_bf16_bits", "quantize", "quantize_block",
-    "dequantize_block", "block_scale_grid", "linear_fwd", "linear_dgrad", "linear_wgrad",
+    "dequantize_block", "block_scale_grid", "linear_fwd", "linear_fwd_gelu", "linear_dgrad", "linear_wgrad",
     "requantize", "gelu_i8", "layernorm_i8", "gelu_f64", "quantization_mse",
 ]
 
@@ -239,6 +239,16 @@ def gelu_i8(q: np.ndarray, s: np.ndarray):
     y = gelu_f64(x).astype(np.float32)
     qo, so = quantize_block(y)
     return qo, so, y
+
+
+def linear_fwd_gelu(Xq, Xs, Wq, Ws, row_blocks=None, col_blocks=None):
+    """Forward with GELU fused into the re-quantization epilogue (the summary's "Approach": the
+    quantization, and here the activation after fc1 as well, happens on chip, before anything is
+    written). Reading: GELU acts on the fp32 pre-activation P that linear_fwd returns, not on its
+    INT8 re-quantization. Returns (P, y) with y = fp32(GELU_f64(P)); requantize() gives the codes
+    of both outputs."""
+    pre = linear_fwd(Xq, Xs, Wq, Ws, row_blocks, col_blocks)
+    return pre, gelu_f64(pre.astype(np.float64)).astype(np.float32)
 
 
 def layernorm_i8(q: np.ndarray, s: np.ndarray, gamma: np.ndarray, beta: np.ndarray,

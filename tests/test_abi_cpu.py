@@ -79,6 +79,15 @@ def test_host_validation_rejects_bad_arguments(lib):
                                jf._Q(1 << 28, 1 << 30, 64, 32), None, None) == -2
     assert lib.jf_linear_wgrad(jf._CQ(1 << 20, 1 << 22, 64, 96), jf._CQ(1 << 24, 1 << 26, 96, 32),
                                jf._Q(1 << 28, 1 << 30, 96, 32), None, None) == -2
+    # fused forward + GELU: the GELU output is required; the pre-activation must not alias it
+    X = jf._CQ(1 << 20, 1 << 22, 64, 96)
+    W = jf._CQ(1 << 24, 1 << 26, 32, 96)
+    none = jf._Q(None, None, 64, 32)
+    assert lib.jf_linear_fwd_gelu(X, W, none, none, None) == -1
+    Y = jf._Q(1 << 28, 1 << 30, 64, 32)
+    assert lib.jf_linear_fwd_gelu(X, W, Y, jf._Q((1 << 28) + 1024, 1 << 31, 64, 32), None) == -5
+    assert lib.jf_linear_fwd_gelu(X, W, Y, jf._Q(1 << 31, 1 << 32, 32, 32), None) == -2
+    assert lib.jf_linear_fwd_gelu(X, jf._CQ(1 << 24, 1 << 26, 32, 64), Y, none, None) == -2
     # LayerNorm needs gamma/beta
     assert lib.jf_layernorm_i8(jf._CQ(1 << 20, 1 << 22, 32, 64), None, fake, ctypes.c_float(1e-5),
                                jf._Q(1 << 28, 1 << 30, 32, 64), None) == -1

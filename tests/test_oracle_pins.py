@@ -334,6 +334,45 @@ def test_gelu_table_and_identities(golden_dir):
     assert O.gelu_f64(np.array([0.0]))[0] == 0.0
 
 
+def test_linear_fwd_gelu_hand_worked_64(golden_dir):
+    """Fused forward + GELU on the hand-worked constant blocks: the large positive blocks pass
+    through GELU unchanged (Phi = 1 in fp64), so their codes and scales are the forward's; the large
+    negative blocks become exactly zero (s = 0, q = 0)."""
+    g = _golden(golden_dir, "gemm_hand_64.json")
+    Aq, As = O.quantize_block(_const_blocks(g["A_scale"], g["A_sign"]))
+    Bq, Bs = O.quantize_block(_const_blocks(g["B_scale"], g["B_sign"]))
+    pre, y = O.linear_fwd_gelu(Aq, As, Bq, Bs)
+    Y = np.array(g["fwd"]["Y"], np.float32)
+    assert np.array_equal(pre, np.kron(Y, np.ones((32, 32), np.float32)))
+    q, s = O.requantize(y)
+    pos = Y > 0
+    assert np.array_equal(s[pos], np.array(g["fwd"]["s"], np.float32)[pos])
+    assert np.all(s[~pos] == 0)
+    exp_q = np.kron(np.where(pos, 127, 0), np.ones((32, 32))).astype(np.int8)
+    assert np.array_equal(q, exp_q)
+
+
+def test_linear_fwd_gelu_normal_cdf_table(golden_dir):
+    """Pre-activations built exactly equal to the table's x (power-of-two scales, one nonzero code
+    per row): the fused output must be x * Phi(x) with Phi from the printed table, which it only is
+    when GELU acts on the fp32 pre-activation (after re-quantization 0.5 would become 32 * 2/127)."""
+    g = _golden(golden_dir, "normal_cdf_table.json")
+    x = np.array(g["x"])
+    Xq = np.zeros((32, 32), np.int8)
+    for i, xv in enumerate(x):
+        assert float(2 * xv).is_integer()                    # x = 0.25 * code * 2 * 1.0 exactly
+        Xq[i, 0] = int(2 * xv)
+    Xs = np.full((1, 1), 0.25, np.float32)
+    Wq = np.zeros((32, 32), np.int8)
+    Wq[:, 0] = 2
+    Ws = np.ones((1, 1), np.float32)
+    pre, y = O.linear_fwd_gelu(Xq, Xs, Wq, Ws)
+    assert np.array_equal(pre[:len(x), 0], x.astype(np.float32))
+    expect = x * np.array(g["Phi"])
+    assert np.allclose(y[:len(x), :].astype(np.float64), expect[:, None], rtol=2.0 ** -23, atol=0)
+    assert np.all(y[len(x):] == 0)
+
+
 def test_gelu_i8_special_blocks():
     # all-zero block -> zero output
     q = np.zeros((32, 64), np.int8)
