@@ -43,7 +43,8 @@ QMAX = 127
 __all__ = [
     "BLOCK", "QMAX", "bf16_bits_to_f32", "f32_to_bf16_bits", "quantize", "quantize_block",
     "dequantize_block", "block_scale_grid", "linear_fwd", "linear_fwd_gelu", "linear_dgrad", "linear_wgrad",
-    "requantize", "gelu_i8", "layernorm_i8", "gelu_f64", "quantization_mse",
+    "requantize", "gelu_i8", "layernorm_i8", "gelu_f64", "quantization_mse", "gelu_grad_f64",
+    "gelu_i8_bwd", "layernorm_i8_bwd",
 ]
 
 
@@ -271,6 +272,49 @@ def layernorm_i8(q: np.ndarray, s: np.ndarray, gamma: np.ndarray, beta: np.ndarr
 # quantization error of a granularity (Jetfire summary, "Measured effects": per-block vs
 # per-token and per-channel quantization error; "Experimental setup": quantization MSE)
 # --------------------------------------------------------------------------------------------
+# --------------------------------------------------------------------------------------------
+# f2: INT8 backward of the non-linear operators (summary, "Approach": every linear and non-linear
+#     operator reads and writes INT8 with per-block scales, the backward pass included)
+# --------------------------------------------------------------------------------------------
+def gelu_grad_f64(x: np.ndarray) -> np.ndarray:
+    """d/dx GELU(x) = Phi(x) + x phi(x) in fp64, with Phi(x) = 0.5 erfc(-x / sqrt 2) and
+    phi(x) = exp(-x^2 / 2) / sqrt(2 pi) the standard normal density."""
+    x = np.asarray(x, np.float64)
+    return 0.5 * _erfc(-x / np.sqrt(2.0)) + x * np.exp(-0.5 * x * x) / np.sqrt(2.0 * np.pi)
+
+
+def gelu_i8_bwd(xq: np.ndarray, xs: np.ndarray, dyq: np.ndarray, dys: np.ndarray):
+    """INT8 backward of GELU_i8. x = fp32(q * s) is the pre-activation, g = fp32(q_dy * s_dy) the
+    upstream gradient; dx = fp32(g * GELU'(x)) with GELU' and the product in fp64, then the
+    per-block quantizer. Returns (q_dx, s_dx, dx_f32)."""
+    x = (np.asarray(xq).astype(np.float32) * block_scale_grid(xs)).astype(np.float32)
+    g = (np.asarray(dyq).astype(np.float32) * block_scale_grid(dys)).astype(np.float32)
+    dx = (g.astype(np.float64) * gelu_grad_f64(x)).astype(np.float32)
+    q, s = quantize_block(dx)
+    return q, s, dx
+
+
+def layernorm_i8_bwd(xq: np.ndarray, xs: np.ndarray, dyq: np.ndarray, dys: np.ndarray,
+                     gamma: np.ndarray, eps: float):
+    """INT8 backward of LayerNorm_i8 (the layer y = (x - mu) rstd gamma + beta of layernorm_i8).
+    x = fp32(q * s) and dy = fp32(q_dy * s_dy); per row, in fp64: mu and the biased variance over
+    the H columns, rstd = 1 / sqrt(var + eps), xhat = (x - mu) rstd, g = dy gamma,
+      dx = rstd (g - mean(g) - xhat mean(g xhat)),
+    and over the rows dgamma = sum dy xhat, dbeta = sum dy. dx is rounded to fp32 and quantized per
+    block; dgamma and dbeta are rounded to fp32. Returns (q_dx, s_dx, dx_f32, dgamma, dbeta)."""
+    x = (np.asarray(xq).astype(np.float32) * block_scale_grid(xs)).astype(np.float64)
+    dy = (np.asarray(dyq).astype(np.float32) * block_scale_grid(dys)).astype(np.float64)
+    mu = x.mean(axis=1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=1, keepdims=True)
+    rstd = 1.0 / np.sqrt(var + np.float64(np.float32(eps)))
+    xhat = (x - mu) * rstd
+    g = dy * np.asarray(gamma, np.float32).astype(np.float64)[None, :]
+    dx = rstd * (g - g.mean(axis=1, keepdims=True) - xhat * (g * xhat).mean(axis=1, keepdims=True))
+    dx32 = dx.astype(np.float32)
+    q, s = quantize_block(dx32)
+    return q, s, dx32, (dy * xhat).sum(axis=0).astype(np.float32), dy.sum(axis=0).astype(np.float32)
+
+
 def quantization_mse(x: np.ndarray, granularity: str) -> float:
     """Mean squared error of quantize -> dequantize for one granularity:
     "block" (32x32), "token" (one scale per row), "channel" (per column), "tensor"."""

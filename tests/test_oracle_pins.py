@@ -427,3 +427,78 @@ def test_layernorm_i8_vs_torch_and_invariants():
     sc = np.full((1, H // 32), 0.25, np.float32)
     _, _, yc = O.layernorm_i8(qc, sc, gamma, beta, 1e-5)
     assert np.array_equal(yc, np.broadcast_to(beta, yc.shape))
+
+
+# ---------------------------------------------------------------------------------------------
+# f2: backward of GELU_i8 and LayerNorm_i8
+# ---------------------------------------------------------------------------------------------
+def test_gelu_grad_against_library_table_and_differences(golden_dir):
+    from scipy.stats import norm
+    xs = np.linspace(-9, 9, 3601)
+    d = O.gelu_grad_f64(xs)
+    # library routines for Phi and phi
+    # (GELU' is O(1); in the far left tail both sides carry the cancellation of Phi + x phi)
+    assert np.allclose(d, norm.cdf(xs) + xs * norm.pdf(xs), rtol=1e-13, atol=1e-16)
+    # the printed normal-CDF table: GELU'(x) - x phi(x) = Phi(x)
+    g = _golden(golden_dir, "normal_cdf_table.json")
+    x = np.array(g["x"])
+    assert np.allclose(O.gelu_grad_f64(x) - x * norm.pdf(x), np.array(g["Phi"]), rtol=1e-14, atol=0)
+    # central differences of the (separately pinned) GELU: a dropped term or a sign error fails
+    h = 1e-5
+    fd = (O.gelu_f64(xs + h) - O.gelu_f64(xs - h)) / (2 * h)
+    assert np.allclose(d, fd, rtol=0, atol=1e-9)
+    assert O.gelu_grad_f64(np.array([0.0]))[0] == 0.5
+
+
+def test_gelu_i8_bwd_special_blocks():
+    rng = np.random.default_rng(21)
+    dyq = rng.integers(-127, 128, size=(32, 96)).astype(np.int8)
+    dyq[0, :] = 127
+    dys = np.array([[1e-3, 2e-3, 4e-3]], np.float32)
+    # x block 0: large positive (GELU' = 1 exactly in fp64), block 1: large negative (GELU' = 0),
+    # block 2: all zero (GELU'(0) = 1/2, exact)
+    xq = np.zeros((32, 96), np.int8)
+    xq[:, :32] = rng.integers(64, 128, size=(32, 32))
+    xq[:, 32:64] = -rng.integers(64, 128, size=(32, 32))
+    xs = np.array([[40.0 / 64, 40.0 / 64, 0.0]], np.float32)
+    q, s, dx = O.gelu_i8_bwd(xq, xs, dyq, dys)
+    g = dyq.astype(np.float32) * O.block_scale_grid(dys)
+    assert np.array_equal(dx[:, :32], g[:, :32])
+    assert np.array_equal(q[:, :32], dyq[:, :32]) and s[0, 0] == dys[0, 0]
+    assert np.all(dx[:, 32:64] == 0) and s[0, 1] == 0 and not q[:, 32:64].any()
+    assert np.array_equal(dx[:, 64:], g[:, 64:] * np.float32(0.5))
+    assert np.array_equal(q[:, 64:], dyq[:, 64:]) and s[0, 2] == dys[0, 2] / 2
+
+
+def test_layernorm_i8_bwd_vs_torch_autograd_and_invariants():
+    rng = np.random.default_rng(22)
+    M, H = 96, 256
+    xq, xs = O.quantize_block(S.activation(rng, M, H, 3, 50.0))
+    dyq, dys = O.quantize_block(S.grad(rng, M, H))
+    gamma = rng.uniform(0.5, 1.5, H).astype(np.float32)
+    beta = rng.normal(0, 0.1, H).astype(np.float32)
+    eps = 1e-5
+    q, s, dx, dgamma, dbeta = O.layernorm_i8_bwd(xq, xs, dyq, dys, gamma, eps)
+    # the library's autograd of layer_norm in fp64, on the same dequantized inputs
+    x = torch.from_numpy((xq.astype(np.float32) * O.block_scale_grid(xs)).astype(np.float64)).requires_grad_()
+    gm = torch.from_numpy(gamma.astype(np.float64)).requires_grad_()
+    bt = torch.from_numpy(beta.astype(np.float64)).requires_grad_()
+    y = torch.nn.functional.layer_norm(x, (H,), gm, bt, eps=float(np.float32(eps)))
+    dy = torch.from_numpy((dyq.astype(np.float32) * O.block_scale_grid(dys)).astype(np.float64))
+    y.backward(dy)
+    ref = x.grad.numpy()
+    assert np.allclose(dx, ref, rtol=2.0 ** -23, atol=1e-7 * np.abs(ref).max())
+    assert np.allclose(dgamma, gm.grad.numpy(), rtol=2.0 ** -23, atol=1e-9 * np.abs(gm.grad.numpy()).max())
+    assert np.allclose(dbeta, bt.grad.numpy(), rtol=2.0 ** -23, atol=0)
+    # requantization is the block quantizer of dx
+    q2, s2 = O.quantize_block(dx)
+    assert np.array_equal(q, q2) and np.array_equal(s, s2)
+    # dx is orthogonal to the constant row (shift invariance of LayerNorm) ...
+    assert np.all(np.abs(ref.sum(1)) <= 1e-9 * np.abs(ref).sum(1))
+    assert np.all(np.abs(dx.astype(np.float64).sum(1)) <= 1e-6 * np.abs(dx).sum(1))
+    # ... and, with eps = 0, to xhat (scale invariance; eps > 0 breaks it by eps / (var + eps))
+    _, _, dx0, _, _ = O.layernorm_i8_bwd(xq, xs, dyq, dys, gamma, 0.0)
+    xd = x.detach().numpy()
+    xh = (xd - xd.mean(1, keepdims=True)) / np.sqrt(xd.var(1, keepdims=True))
+    dx0 = dx0.astype(np.float64)
+    assert np.all(np.abs((dx0 * xh).sum(1)) <= 1e-6 * np.abs(dx0 * xh).sum(1))
