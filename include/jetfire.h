@@ -5,7 +5,7 @@
  * Data Flow and Per-Block Quantization", atlas.scime.ai summary page, section "Approach"):
  * every linear and non-linear operator of a transformer layer reads and writes INT8 tensors that
  * carry one scale factor per block, with block size B = 32; quantization is applied on-chip, and
- * the weight gradient is also computed in INT8 with per-block scales. The "Fp8 vs int8" page gives
+ * the weight gradient, too, is an INT8 product with per-block scales. The "Fp8 vs int8" page gives
  * the signed INT8 range and the dequantization x = FP(q) * s.
  *
  * Readings taken where the pages are silent (each is stated once here and applies to every call):
@@ -76,7 +76,8 @@ typedef enum {
   JF_ERR_ALIAS = -5,   /* an output overlaps an input */
   JF_ERR_CUDA = -6,    /* a CUDA runtime or driver call failed (launch, tensor-map encode) */
   JF_ERR_TIMEOUT = -7, /* reported by jf_device_status: a kernel's bounded wait ran out */
-  JF_ERR_DEVICE = -8   /* no usable sm_100 device is current */
+  JF_ERR_DEVICE = -8,  /* no usable sm_100 device is current */
+  JF_ERR_WORKSPACE = -9 /* the caller's workspace is NULL, misaligned or smaller than required */
 } jf_status;
 
 /*
@@ -132,8 +133,8 @@ JF_API int jf_linear_fwd_gelu(jf_cqtensor X, jf_cqtensor W, jf_qtensor Y, jf_qte
 JF_API int jf_linear_dgrad(jf_cqtensor dY, jf_cqtensor W, jf_qtensor dX, float* dx_f32, void* stream);
 
 /*
- * a5. Weight gradient dW = dY^T X (summary, "Approach": "the weight gradient is also computed in
- *     INT8 with per-block scales").
+ * a5. Weight gradient dW = dY^T X (summary, "Approach": the weight gradient, too, is an INT8
+ *     product with one scale per block).
  *   dY [M, N], X [M, K] (both read re-blocked along M), dW [N, K] (output).
  *   dW(n, k) = sum_mb fp32(sdY(mb, n/32) sX(mb, k/32)) * sum_{m in mb} dYq(m, n) Xq(m, k).
  *   dw_f32 as y_f32 above (an optimizer, or a data-parallel gradient reduction, wants fp32).
@@ -153,6 +154,37 @@ JF_API int jf_gelu_i8(jf_cqtensor X, jf_qtensor Y, void* stream);
  */
 JF_API int jf_layernorm_i8(jf_cqtensor X, const float* gamma, const float* beta, float eps, jf_qtensor Y,
                     void* stream);
+
+/*
+ * f2. Backward of GELU_i8 (summary, "Approach": the backward pass keeps the INT8 data flow too).
+ *   X   [M, N] the saved pre-activation (the forward's input), dY [M, N] the upstream gradient,
+ *   dX  [M, N] output: requant(fp32(dY.q) dY.s * GELU'(fp32(X.q) X.s)) per 32x32 block, where
+ *       GELU'(x) = Phi(x) + x phi(x) (Phi, phi: the standard normal CDF and density).
+ *   Errors: JF_ERR_SHAPE if the three shapes differ; JF_ERR_ALIAS if dX overlaps an input.
+ */
+JF_API int jf_gelu_i8_bwd(jf_cqtensor X, jf_cqtensor dY, jf_qtensor dX, void* stream);
+
+/*
+ * f2. Backward of LayerNorm_i8 (same layer as jf_layernorm_i8, same eps).
+ *   X      [M, H] the forward's input; dY [M, H] the upstream gradient; gamma fp32 [H] (16-byte
+ *          aligned). Per row, with x = fp32(q) s, xhat = (x - mean) rstd, rstd = 1 / sqrt(var + eps)
+ *          and g = dy gamma:
+ *            dX = requant(rstd (g - mean(g) - xhat mean(g xhat))) per 32x32 block,
+ *          and over all rows dgamma = sum dy xhat, dbeta = sum dy (fp32 [H], deterministic).
+ *   dgamma, dbeta  nullable device fp32 [H]; when either is given, `workspace` must hold at least
+ *          jf_layernorm_i8_bwd_workspace_bytes(M, H) bytes of caller-owned device memory, 16-byte
+ *          aligned (per-strip column sums; its contents on entry do not matter). Otherwise the
+ *          workspace is not used and may be NULL.
+ *   Errors: JF_ERR_NULL if gamma or dX.q is NULL; JF_ERR_WORKSPACE as above; JF_ERR_ALIAS if any
+ *          output (workspace included) overlaps an input or another output.
+ */
+JF_API int jf_layernorm_i8_bwd(jf_cqtensor X, jf_cqtensor dY, const float* gamma, float eps, jf_qtensor dX,
+                               float* dgamma, float* dbeta, void* workspace, int64_t workspace_bytes,
+                               void* stream);
+
+/* Bytes of workspace jf_layernorm_i8_bwd needs for X of [rows, cols]: (rows / 32) * 2 * cols * 4,
+ * or -1 for an invalid shape. */
+JF_API int64_t jf_layernorm_i8_bwd_workspace_bytes(int64_t rows, int64_t cols);
 
 /* Static description of a status code (never NULL). */
 JF_API const char* jf_strerror(int status);

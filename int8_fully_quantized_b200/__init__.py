@@ -24,7 +24,9 @@ from .build_lib import LIB_PATH
 __all__ = [
     "QTensor", "JetfireError", "load_library", "empty_qtensor", "jf_quantize_block", "jf_dequantize_block",
     "jf_linear_fwd", "jf_linear_fwd_gelu", "jf_linear_dgrad", "jf_linear_wgrad", "jf_gelu_i8", "jf_layernorm_i8",
-    "jf_strerror", "jf_device_status", "jf_sm_count", "quantize_block", "dequantize_block", "linear_fwd",
+    "jf_gelu_i8_bwd", "jf_layernorm_i8_bwd", "jf_layernorm_i8_bwd_workspace_bytes", "gelu_i8_bwd",
+    "layernorm_i8_bwd", "jf_strerror", "jf_device_status", "jf_sm_count", "quantize_block", "dequantize_block",
+    "linear_fwd",
     "linear_fwd_gelu", "linear_dgrad",
     "linear_wgrad", "gelu_i8", "layernorm_i8", "EXPORTED_SYMBOLS", "JF_F32", "JF_BF16", "JF_F16",
 ]
@@ -35,7 +37,8 @@ _DTYPES = {torch.float32: JF_F32, torch.bfloat16: JF_BF16, torch.float16: JF_F16
 EXPORTED_SYMBOLS = (
     "jf_quantize_block", "jf_dequantize_block", "jf_linear_fwd", "jf_linear_fwd_gelu", "jf_linear_dgrad",
     "jf_linear_wgrad",
-    "jf_gelu_i8", "jf_layernorm_i8", "jf_strerror", "jf_device_status", "jf_sm_count",
+    "jf_gelu_i8", "jf_layernorm_i8", "jf_gelu_i8_bwd", "jf_layernorm_i8_bwd", "jf_layernorm_i8_bwd_workspace_bytes",
+    "jf_strerror", "jf_device_status", "jf_sm_count",
 )
 
 
@@ -76,6 +79,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.jf_linear_fwd_gelu.argtypes = [_CQ, _CQ, _Q, _Q, vp]
     lib.jf_gelu_i8.argtypes = [_CQ, _Q, vp]
     lib.jf_layernorm_i8.argtypes = [_CQ, vp, vp, ctypes.c_float, _Q, vp]
+    lib.jf_gelu_i8_bwd.argtypes = [_CQ, _CQ, _Q, vp]
+    lib.jf_layernorm_i8_bwd.argtypes = [_CQ, _CQ, vp, ctypes.c_float, _Q, vp, vp, vp, i64, vp]
+    lib.jf_layernorm_i8_bwd_workspace_bytes.argtypes = [i64, i64]
     lib.jf_strerror.argtypes = [i32]
     lib.jf_strerror.restype = ctypes.c_char_p
     lib.jf_device_status.argtypes = [vp]
@@ -83,6 +89,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     for name in EXPORTED_SYMBOLS:
         if name != "jf_strerror":
             getattr(lib, name).restype = ctypes.c_int
+    lib.jf_layernorm_i8_bwd_workspace_bytes.restype = i64
     _lib = lib
     return lib
 
@@ -189,6 +196,25 @@ def jf_layernorm_i8(X: QTensor, gamma: torch.Tensor, beta: torch.Tensor, eps: fl
                                _stream(stream)), "jf_layernorm_i8")
 
 
+def jf_gelu_i8_bwd(X: QTensor, dY: QTensor, dX: QTensor, stream=None) -> None:
+    lib = load_library()
+    _check(lib.jf_gelu_i8_bwd(_cq(X), _cq(dY), _q(dX, X.rows, X.cols), _stream(stream)), "jf_gelu_i8_bwd")
+
+
+def jf_layernorm_i8_bwd_workspace_bytes(rows: int, cols: int) -> int:
+    return int(load_library().jf_layernorm_i8_bwd_workspace_bytes(rows, cols))
+
+
+def jf_layernorm_i8_bwd(X: QTensor, dY: QTensor, gamma: torch.Tensor, eps: float, dX: QTensor,
+                        dgamma: Optional[torch.Tensor] = None, dbeta: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    lib = load_library()
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.jf_layernorm_i8_bwd(_cq(X), _cq(dY), _ptr(gamma), ctypes.c_float(eps), _q(dX, X.rows, X.cols),
+                                   _ptr(dgamma), _ptr(dbeta), _ptr(workspace), nbytes, _stream(stream)),
+           "jf_layernorm_i8_bwd")
+
+
 def jf_strerror(status: int) -> str:
     return load_library().jf_strerror(int(status)).decode()
 
@@ -248,6 +274,23 @@ def gelu_i8(X: QTensor, stream=None) -> QTensor:
     Y = empty_qtensor(X.rows, X.cols, X.q.device)
     jf_gelu_i8(X, Y, stream)
     return Y
+
+
+def gelu_i8_bwd(X: QTensor, dY: QTensor, stream=None) -> QTensor:
+    """dX = requant(dY * GELU'(X)) on INT8 blocks; X is the saved pre-activation."""
+    dX = empty_qtensor(X.rows, X.cols, X.q.device)
+    jf_gelu_i8_bwd(X, dY, dX, stream)
+    return dX
+
+
+def layernorm_i8_bwd(X: QTensor, dY: QTensor, gamma: torch.Tensor, eps: float = 1e-5, stream=None):
+    """(dX, dgamma, dbeta) of LayerNorm_i8; the workspace is allocated here, per call."""
+    dX = empty_qtensor(X.rows, X.cols, X.q.device)
+    dgamma = torch.empty(X.cols, dtype=torch.float32, device=X.q.device)
+    dbeta = torch.empty_like(dgamma)
+    ws = torch.empty(jf_layernorm_i8_bwd_workspace_bytes(X.rows, X.cols), dtype=torch.uint8, device=X.q.device)
+    jf_layernorm_i8_bwd(X, dY, gamma, eps, dX, dgamma, dbeta, ws, stream)
+    return dX, dgamma, dbeta
 
 
 def layernorm_i8(X: QTensor, gamma: torch.Tensor, beta: torch.Tensor, eps: float = 1e-5, stream=None) -> QTensor:

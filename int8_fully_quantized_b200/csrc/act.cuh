@@ -8,4 +8,10 @@ namespace jf {
 // accuracy, while erfc keeps it.
 __device__ __forceinline__ float gelu_f32(float x) { return 0.5f * x * erfcf(x * -0.70710678118654752440f); }
 
+// GELU'(x) = Phi(x) + x phi(x), with Phi(x) = 0.5 erfc(-x / sqrt 2) and phi(x) = exp(-x^2 / 2) / sqrt(2 pi).
+// For x -> -inf both terms vanish (the sum is about phi(x) (1/|x| - |x|), no cancellation that matters).
+__device__ __forceinline__ float gelu_grad_f32(float x) {
+  return fmaf(x * 0.39894228040143267794f, expf(-0.5f * x * x), 0.5f * erfcf(x * -0.70710678118654752440f));
+}
+
 }  // namespace jf

@@ -244,6 +244,64 @@ int jf_layernorm_i8(jf_cqtensor X, const float* gamma, const float* beta, float 
       jf::launch_layernorm_i8(X.q, X.s, X.rows, X.cols, gamma, beta, eps, Y.q, Y.s, static_cast<cudaStream_t>(stream)));
 }
 
+int jf_gelu_i8_bwd(jf_cqtensor X, jf_cqtensor dY, jf_qtensor dX, void* stream) {
+  int st;
+  if ((st = check_cq(X)) != JF_OK) return st;
+  if ((st = check_cq(dY)) != JF_OK) return st;
+  if ((st = check_q(dX, true)) != JF_OK) return st;
+  if (X.rows != dY.rows || X.cols != dY.cols || X.rows != dX.rows || X.cols != dX.cols) return JF_ERR_SHAPE;
+  if (X.rows == 0 || X.cols == 0) return JF_OK;
+  const int64_t nq = qbytes(X), ns = sbytes(X.rows, X.cols);
+  const void* ins[4] = {X.q, X.s, dY.q, dY.s};
+  const int64_t in_n[4] = {nq, ns, nq, ns};
+  for (int i = 0; i < 4; ++i)
+    if (overlap(dX.q, nq, ins[i], in_n[i]) || overlap(dX.s, ns, ins[i], in_n[i])) return JF_ERR_ALIAS;
+  if (overlap(dX.q, nq, dX.s, ns)) return JF_ERR_ALIAS;
+  const DevInfo d = device_info();
+  if (!d.ok) return JF_ERR_DEVICE;
+  return cuda_status(jf::launch_gelu_i8_bwd(X.q, X.s, dY.q, dY.s, X.rows, X.cols, dX.q, dX.s, d.sm_count,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+int64_t jf_layernorm_i8_bwd_workspace_bytes(int64_t rows, int64_t cols) {
+  if (!dims_ok(rows, cols)) return -1;
+  return (rows / 32) * 2 * cols * 4;
+}
+
+int jf_layernorm_i8_bwd(jf_cqtensor X, jf_cqtensor dY, const float* gamma, float eps, jf_qtensor dX, float* dgamma,
+                        float* dbeta, void* workspace, int64_t workspace_bytes, void* stream) {
+  int st;
+  if ((st = check_cq(X)) != JF_OK) return st;
+  if ((st = check_cq(dY)) != JF_OK) return st;
+  if ((st = check_q(dX, true)) != JF_OK) return st;
+  if (X.rows != dY.rows || X.cols != dY.cols || X.rows != dX.rows || X.cols != dX.cols) return JF_ERR_SHAPE;
+  if (X.rows == 0 || X.cols == 0) return JF_OK;
+  if (gamma == nullptr) return JF_ERR_NULL;
+  if (!aligned(gamma, 16) || !aligned(dgamma, 4) || !aligned(dbeta, 4)) return JF_ERR_ALIGN;
+  const bool want_param_grads = dgamma != nullptr || dbeta != nullptr;
+  if (want_param_grads &&
+      (workspace == nullptr || !aligned(workspace, 16) ||
+       workspace_bytes < jf_layernorm_i8_bwd_workspace_bytes(X.rows, X.cols)))
+    return JF_ERR_WORKSPACE;
+  const int64_t nq = qbytes(X), ns = sbytes(X.rows, X.cols), H = X.cols;
+  const int64_t nw = want_param_grads ? jf_layernorm_i8_bwd_workspace_bytes(X.rows, X.cols) : 0;
+  const void* ins[5] = {X.q, X.s, dY.q, dY.s, gamma};
+  const int64_t in_n[5] = {nq, ns, nq, ns, H * 4};
+  const void* outs[5] = {dX.q, dX.s, dgamma, dbeta, want_param_grads ? workspace : nullptr};
+  const int64_t out_n[5] = {nq, ns, H * 4, H * 4, nw};
+  for (int o = 0; o < 5; ++o) {
+    for (int i = 0; i < 5; ++i)
+      if (overlap(outs[o], out_n[o], ins[i], in_n[i])) return JF_ERR_ALIAS;
+    for (int o2 = o + 1; o2 < 5; ++o2)
+      if (overlap(outs[o], out_n[o], outs[o2], out_n[o2])) return JF_ERR_ALIAS;
+  }
+  const DevInfo d = device_info();
+  if (!d.ok) return JF_ERR_DEVICE;
+  return cuda_status(jf::launch_layernorm_i8_bwd(X.q, X.s, dY.q, dY.s, X.rows, X.cols, gamma, eps, dX.q, dX.s,
+                                                 want_param_grads ? static_cast<float*>(workspace) : nullptr,
+                                                 dgamma, dbeta, static_cast<cudaStream_t>(stream)));
+}
+
 const char* jf_strerror(int status) {
   switch (status) {
     case JF_OK: return "ok";
@@ -255,6 +313,7 @@ const char* jf_strerror(int status) {
     case JF_ERR_CUDA: return "a CUDA runtime/driver call failed";
     case JF_ERR_TIMEOUT: return "a kernel's bounded wait timed out; outputs are undefined";
     case JF_ERR_DEVICE: return "no usable sm_100 (B200) device is current";
+    case JF_ERR_WORKSPACE: return "workspace is NULL, not 16-byte aligned or smaller than the size asked for";
     default: return "unknown status";
   }
 }

@@ -1,0 +1,283 @@
+// INT8 backward of the non-linear operators on 32x32 blocks: GELU_i8 and LayerNorm_i8.
+//
+// Jetfire (atlas.scime.ai summary, "Approach"): every linear and non-linear operator of the
+// transformer block reads and writes INT8 tensors with one scale per 32x32 block, in the backward
+// pass as in the forward. Both kernels here are memory-bound: they read two INT8 tensors (the
+// saved forward input and the upstream gradient) and write one, re-quantized per block on chip.
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "act.cuh"
+#include "kernels.h"
+#include "ptx.cuh"
+#include "quant.cuh"
+
+namespace jf {
+
+// ---------------------------------------------------------------------------------------------
+// GELU_i8 backward: dx = fp32(dy) * GELU'(fp32(x)) per element, re-quantized per block. One warp
+// per block, lane l takes columns 16 (l % 2) .. +15 of rows l / 2 and 16 + l / 2 (two 16-byte
+// chunks per tensor). A block of x has at most 255 distinct values q * s, so the warp tabulates
+// GELU' of all of them first (8 evaluations per lane instead of 32) and looks its values up.
+// ---------------------------------------------------------------------------------------------
+constexpr int kGeluBwdWarps = 8;
+
+__global__ void __launch_bounds__(32 * kGeluBwdWarps, 3) gelu_i8_bwd_kernel(
+    const int8_t* __restrict__ xq, const float* __restrict__ xs, const int8_t* __restrict__ dq,
+    const float* __restrict__ ds, int64_t R, int64_t C, int8_t* __restrict__ qo, float* __restrict__ so) {
+  __shared__ float table[kGeluBwdWarps][256];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  float* tab = table[wib];
+  const int64_t nbc = C >> 5;
+  const int64_t nblocks = (R >> 5) * nbc;
+  const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
+  const int r0 = lane >> 1, c0 = (lane & 1) * 16;
+  for (int64_t b = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; b < nblocks; b += nwarps) {
+    const int64_t bi = b / nbc, bj = b - bi * nbc;
+    const float sx = __ldg(xs + b), sd = __ldg(ds + b);
+    const int64_t off = (bi * 32 + r0) * C + bj * 32 + c0;
+    const uint4 a0 = ld_stream_v4(xq + off);
+    const uint4 a1 = ld_stream_v4(xq + off + 16 * C);
+    const uint4 d0 = ld_stream_v4(dq + off);
+    const uint4 d1 = ld_stream_v4(dq + off + 16 * C);
+    // table[u] = GELU'(fp32(u - 128) * sx) for the code u - 128
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int u = lane + 32 * j;
+      tab[u] = gelu_grad_f32(float(u - 128) * sx);
+    }
+    __syncwarp();
+    const uint32_t wx[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const uint32_t wd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+    float v[32];
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t u = wx[i] ^ 0x80808080u;  // code + 128 in each byte
+      float g[4];
+      i8x4_to_f32(wd[i], g);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[4 * i + j] = (g[j] * sd) * tab[(u >> (8 * j)) & 0xFFu];
+        m = fmaxf(m, fabsf(v[4 * i + j]));
+      }
+    }
+    __syncwarp();  // the table is rewritten for the next block only after every lane has read it
+    const BlockQuant bq = block_quant(warp_max_nonneg(m));
+    uint32_t o[8];
+    quant_pack<32>(v, bq, o);
+    *reinterpret_cast<uint4*>(qo + off) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(qo + off + 16 * C) = make_uint4(o[4], o[5], o[6], o[7]);
+    if (lane == 0) so[b] = bq.s;
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// LayerNorm_i8 backward. For the layer y = (x - mu) rstd gamma + beta (mu, biased variance over the
+// H columns of a row, rstd = 1 / sqrt(var + eps)), with xhat = (x - mu) rstd and g = dy gamma:
+//   dx = rstd (g - mean(g) - xhat mean(g xhat)),  dgamma = sum_rows dy xhat,  dbeta = sum_rows dy.
+// One CTA of 8 warps per 32-row strip, three CTAs per SM:
+//   phase 1: warp w reduces rows w, w + 8, w + 16 and w + 24, each in one pass: sums of x, x^2, g and g x (chunk partials
+//            of 16 values in fp32, accumulated in fp64). Then mean, rstd, mean(g) and
+//            mean(g xhat) = rstd (mean(g x) - mean * mean(g)) per row, kept in shared memory.
+//   phase 2: warp w handles column blocks w, w + 8, ...: lane l takes the 4 columns 4 (l % 8) .. +3
+//            of rows l / 8 + 4 i (i = 0..7), computes dx, re-quantizes the block and sums dy xhat
+//            and dy of its columns over the strip's 32 rows (shuffles across the 4 row groups).
+//            The strip (2 x 32 H bytes) is read a second time, from L2.
+//   The per-strip column sums go to part[strip][0 | 1][H] when gamma or beta gradients are asked
+//   for; ln_bwd_reduce_kernel then adds them over the strips in a fixed order (deterministic).
+// ---------------------------------------------------------------------------------------------
+constexpr int kLnbThreads = 256;
+
+__global__ void __launch_bounds__(kLnbThreads, 3) layernorm_i8_bwd_kernel(
+    const int8_t* __restrict__ xq, const float* __restrict__ xs, const int8_t* __restrict__ dq,
+    const float* __restrict__ ds, int64_t R, int64_t H, const float* __restrict__ gamma, float eps,
+    int8_t* __restrict__ qo, float* __restrict__ so, float* __restrict__ part) {
+  __shared__ float4 s_stat[32];  // per row: mean, rstd, mean(g), mean(g xhat)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t strip = blockIdx.x;
+  const int64_t nbc = H >> 5;
+  const int8_t* xstrip = xq + strip * 32 * H;
+  const int8_t* dstrip = dq + strip * 32 * H;
+  const float* xss = xs + strip * nbc;
+  const float* dss = ds + strip * nbc;
+  for (int rw = warp; rw < 32; rw += kLnbThreads / 32) {
+    const int8_t* xrow = xstrip + int64_t(rw) * H;
+    const int8_t* drow = dstrip + int64_t(rw) * H;
+    double sum_x = 0.0, sum_xx = 0.0, sum_g = 0.0, sum_gx = 0.0;
+    constexpr int kUnroll = 4;  // 16-byte chunks of each tensor a lane keeps in flight
+    for (int64_t ch0 = lane; ch0 < (H >> 4); ch0 += 32 * kUnroll) {
+      uint4 av[kUnroll], dv[kUnroll];
+      float scx[kUnroll], scd[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t ch = ch0 + 32 * u;
+        if (ch < (H >> 4)) {
+          av[u] = ld_stream_v4(xrow + ch * 16);
+          dv[u] = ld_stream_v4(drow + ch * 16);
+          scx[u] = __ldg(xss + (ch >> 1));
+          scd[u] = __ldg(dss + (ch >> 1));
+        } else {
+          av[u] = dv[u] = make_uint4(0u, 0u, 0u, 0u);
+          scx[u] = scd[u] = 0.0f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t ch = ch0 + 32 * u;
+        if (ch >= (H >> 4)) break;
+        const uint32_t wx[4] = {av[u].x, av[u].y, av[u].z, av[u].w};
+        const uint32_t wd[4] = {dv[u].x, dv[u].y, dv[u].z, dv[u].w};
+        const float4* g4 = reinterpret_cast<const float4*>(gamma + ch * 16);
+        float px = 0.0f, pxx = 0.0f, pg = 0.0f, pgx = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 gm = __ldg(g4 + i);
+          const float gmv[4] = {gm.x, gm.y, gm.z, gm.w};
+          float fx[4], fd[4];
+          i8x4_to_f32(wx[i], fx);
+          i8x4_to_f32(wd[i], fd);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float x = fx[j] * scx[u];
+            const float g = (fd[j] * scd[u]) * gmv[j];
+            px += x;
+            pxx = fmaf(x, x, pxx);
+            pg += g;
+            pgx = fmaf(g, x, pgx);
+          }
+        }
+        sum_x += double(px);
+        sum_xx += double(pxx);
+        sum_g += double(pg);
+        sum_gx += double(pgx);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      sum_x += __shfl_xor_sync(0xffffffffu, sum_x, o);
+      sum_xx += __shfl_xor_sync(0xffffffffu, sum_xx, o);
+      sum_g += __shfl_xor_sync(0xffffffffu, sum_g, o);
+      sum_gx += __shfl_xor_sync(0xffffffffu, sum_gx, o);
+    }
+    if (lane == 0) {
+      const double inv_h = 1.0 / double(H);
+      const double mean = sum_x * inv_h;
+      double var = sum_xx * inv_h - mean * mean;
+      var = var > 0.0 ? var : 0.0;
+      const double rstd = 1.0 / sqrt(var + double(eps));
+      const double mg = sum_g * inv_h;
+      const double mgx = rstd * (sum_gx * inv_h - mean * mg);
+      s_stat[rw] = make_float4(float(mean), float(rstd), float(mg), float(mgx));
+    }
+  }
+  __syncthreads();
+  const int cg = lane & 7, rg = lane >> 3;
+  for (int64_t bj = warp; bj < nbc; bj += kLnbThreads / 32) {
+    const float sx = __ldg(xss + bj), sd = __ldg(dss + bj);
+    const int64_t col = bj * 32 + 4 * cg;
+    const float4 gm4 = __ldg(reinterpret_cast<const float4*>(gamma + col));
+    const float gm[4] = {gm4.x, gm4.y, gm4.z, gm4.w};
+    uint32_t wx[8], wd[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int64_t off = int64_t(rg + 4 * i) * H + col;
+      wx[i] = ld_stream_b32(xstrip + off);
+      wd[i] = ld_stream_b32(dstrip + off);
+    }
+    float v[32], pgam[4] = {0.0f, 0.0f, 0.0f, 0.0f}, pbet[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float fx[4], fd[4];
+      i8x4_to_f32(wx[i], fx);
+      i8x4_to_f32(wd[i], fd);
+      const float4 st = s_stat[rg + 4 * i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float xhat = (fx[j] * sx - st.x) * st.y;
+        const float dy = fd[j] * sd;
+        const float dx = st.y * (fmaf(dy, gm[j], -st.z) - xhat * st.w);
+        v[4 * i + j] = dx;
+        m = fmaxf(m, fabsf(dx));
+        pgam[j] = fmaf(dy, xhat, pgam[j]);
+        pbet[j] += dy;
+      }
+    }
+    const BlockQuant bq = block_quant(warp_max_nonneg(m));
+    uint32_t o[8];
+    quant_pack<32>(v, bq, o);
+    int8_t* dst = qo + strip * 32 * H;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) *reinterpret_cast<uint32_t*>(dst + int64_t(rg + 4 * i) * H + col) = o[i];
+    if (lane == 0) so[strip * nbc + bj] = bq.s;
+    if (part != nullptr) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        pgam[j] += __shfl_xor_sync(0xffffffffu, pgam[j], 8);
+        pgam[j] += __shfl_xor_sync(0xffffffffu, pgam[j], 16);
+        pbet[j] += __shfl_xor_sync(0xffffffffu, pbet[j], 8);
+        pbet[j] += __shfl_xor_sync(0xffffffffu, pbet[j], 16);
+      }
+      if (rg == 0) {
+        float* pg = part + strip * 2 * H;
+        *reinterpret_cast<float4*>(pg + col) = make_float4(pgam[0], pgam[1], pgam[2], pgam[3]);
+        *reinterpret_cast<float4*>(pg + H + col) = make_float4(pbet[0], pbet[1], pbet[2], pbet[3]);
+      }
+    }
+  }
+}
+
+// dgamma[c] and dbeta[c] = sums over the strips of part[strip][0 | 1][c], in fp64 and in a fixed
+// order (warp w adds strips w, w + 8, ...; the 8 warp sums are then added in warp order), so the
+// result does not depend on scheduling. One CTA per 32 columns, lane = column.
+__global__ void __launch_bounds__(256) ln_bwd_reduce_kernel(const float* __restrict__ part, int64_t nstrips,
+                                                            int64_t H, float* __restrict__ dgamma,
+                                                            float* __restrict__ dbeta) {
+  __shared__ double sg[8][32], sb[8][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t col = int64_t(blockIdx.x) * 32 + lane;
+  double ag = 0.0, ab = 0.0;
+  for (int64_t st = warp; st < nstrips; st += 8) {
+    ag += double(part[st * 2 * H + col]);
+    ab += double(part[st * 2 * H + H + col]);
+  }
+  sg[warp][lane] = ag;
+  sb[warp][lane] = ab;
+  __syncthreads();
+  if (warp == 0) {
+    double tg = 0.0, tb = 0.0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      tg += sg[w][lane];
+      tb += sb[w][lane];
+    }
+    if (dgamma != nullptr) dgamma[col] = float(tg);
+    if (dbeta != nullptr) dbeta[col] = float(tb);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------------------------
+cudaError_t launch_gelu_i8_bwd(const int8_t* xq, const float* xs, const int8_t* dq, const float* ds, int64_t R,
+                               int64_t C, int8_t* qo, float* so, int sm_count, cudaStream_t st) {
+  const int64_t nblocks = (R / 32) * (C / 32);
+  int64_t grid = (nblocks + kGeluBwdWarps - 1) / kGeluBwdWarps;
+  const int64_t cap = int64_t(sm_count) * 8;
+  if (grid > cap) grid = cap;
+  gelu_i8_bwd_kernel<<<int(grid < 1 ? 1 : grid), 32 * kGeluBwdWarps, 0, st>>>(xq, xs, dq, ds, R, C, qo, so);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_layernorm_i8_bwd(const int8_t* xq, const float* xs, const int8_t* dq, const float* ds, int64_t R,
+                                    int64_t H, const float* gamma, float eps, int8_t* qo, float* so, float* part,
+                                    float* dgamma, float* dbeta, cudaStream_t st) {
+  layernorm_i8_bwd_kernel<<<int(R / 32), kLnbThreads, 0, st>>>(xq, xs, dq, ds, R, H, gamma, eps, qo, so, part);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || part == nullptr) return e;
+  ln_bwd_reduce_kernel<<<int(H / 32), 256, 0, st>>>(part, R / 32, H, dgamma, dbeta);
+  return cudaGetLastError();
+}
+
+}  // namespace jf

@@ -12,6 +12,13 @@ cudaError_t launch_dequantize(const int8_t* q, const float* s, int64_t R, int64_
                               int sm_count, cudaStream_t st);
 cudaError_t launch_gelu_i8(const int8_t* q, const float* s, int64_t R, int64_t C, int8_t* qo, float* so,
                            int sm_count, cudaStream_t st);
+// INT8 backward of GELU_i8 and LayerNorm_i8 (backward.cu). `part` is the [R/32][2][H] fp32
+// workspace of per-strip column sums; null when neither dgamma nor dbeta is wanted.
+cudaError_t launch_gelu_i8_bwd(const int8_t* xq, const float* xs, const int8_t* dq, const float* ds, int64_t R,
+                               int64_t C, int8_t* qo, float* so, int sm_count, cudaStream_t st);
+cudaError_t launch_layernorm_i8_bwd(const int8_t* xq, const float* xs, const int8_t* dq, const float* ds, int64_t R,
+                                    int64_t H, const float* gamma, float eps, int8_t* qo, float* so, float* part,
+                                    float* dgamma, float* dbeta, cudaStream_t st);
 cudaError_t launch_layernorm_i8(const int8_t* q, const float* s, int64_t R, int64_t H, const float* gamma,
                                 const float* beta, float eps, int8_t* qo, float* so, cudaStream_t st);
 

@@ -21,7 +21,7 @@ def lib():
 
 def _declared():
     text = open(os.path.join(ROOT, "include", "jetfire.h")).read()
-    return sorted(set(re.findall(r"^\s*(?:JF_API\s+)?(?:int|const char\s*\*)\s+(jf_\w+)\s*\(", text, flags=re.M)))
+    return sorted(set(re.findall(r"^\s*(?:JF_API\s+)?(?:int|int64_t|const char\s*\*)\s+(jf_\w+)\s*\(", text, flags=re.M)))
 
 
 def test_header_declares_the_entry_points():
@@ -88,6 +88,24 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert lib.jf_linear_fwd_gelu(X, W, Y, jf._Q((1 << 28) + 1024, 1 << 31, 64, 32), None) == -5
     assert lib.jf_linear_fwd_gelu(X, W, Y, jf._Q(1 << 31, 1 << 32, 32, 32), None) == -2
     assert lib.jf_linear_fwd_gelu(X, jf._CQ(1 << 24, 1 << 26, 32, 64), Y, none, None) == -2
+    # backward of GELU: shapes must agree, dX must not alias an input
+    Xc = jf._CQ(1 << 20, 1 << 22, 64, 96)
+    assert lib.jf_gelu_i8_bwd(Xc, jf._CQ(1 << 24, 1 << 26, 64, 64), jf._Q(1 << 28, 1 << 30, 64, 96), None) == -2
+    assert lib.jf_gelu_i8_bwd(Xc, jf._CQ(1 << 24, 1 << 26, 64, 96), jf._Q((1 << 24) + 32, 1 << 30, 64, 96),
+                              None) == -5
+    # backward of LayerNorm: workspace size, presence and alignment
+    need = lib.jf_layernorm_i8_bwd_workspace_bytes(64, 96)
+    assert need == 2 * 2 * 96 * 4 and lib.jf_layernorm_i8_bwd_workspace_bytes(33, 96) == -1
+    dYc = jf._CQ(1 << 24, 1 << 26, 64, 96)
+    dXq = jf._Q(1 << 28, 1 << 30, 64, 96)
+    g, dg, db, ws = vp(1 << 32), vp(1 << 33), vp(1 << 34), vp(1 << 35)
+    f = ctypes.c_float(1e-5)
+    assert lib.jf_layernorm_i8_bwd(Xc, dYc, g, f, dXq, dg, db, None, 0, None) == -9
+    assert lib.jf_layernorm_i8_bwd(Xc, dYc, g, f, dXq, dg, db, ws, need - 4, None) == -9
+    assert lib.jf_layernorm_i8_bwd(Xc, dYc, g, f, dXq, dg, db, vp((1 << 35) + 4), need, None) == -9
+    assert lib.jf_layernorm_i8_bwd(Xc, dYc, None, f, dXq, dg, db, ws, need, None) == -1
+    assert lib.jf_layernorm_i8_bwd(Xc, dYc, g, f, dXq, dg, vp((1 << 33) + 8), ws, need, None) == -5
+    assert lib.jf_layernorm_i8_bwd(Xc, dYc, g, f, dXq, dg, db, vp((1 << 34) + 16), need, None) == -5
     # LayerNorm needs gamma/beta
     assert lib.jf_layernorm_i8(jf._CQ(1 << 20, 1 << 22, 32, 64), None, fake, ctypes.c_float(1e-5),
                                jf._Q(1 << 28, 1 << 30, 32, 64), None) == -1
