@@ -36,7 +36,7 @@ if ROOT not in sys.path:
 METRIC = "per-block INT8 GEMM TOPS (% INT8 peak); quantize/GELU/LN GB/s (% HBM)"
 WORKLOAD = "gpt2m_fc1"
 NOMINAL_I8_OVER_BF16 = 2.0       # dense int8 (4.5 POPS) / dense bf16 (2.25 PFLOP/s), nominal B200
-FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 
 
 def parse_args():
@@ -51,8 +51,13 @@ def parse_args():
     p.add_argument("--sweep", action="store_true",
                    help="time the memory-bound kernels on the M x 4096 sweep instead of the step")
     p.add_argument("--sweep-m", type=int, nargs="*", default=[1024, 8192, 65536])
-    p.add_argument("--sweep-ops", nargs="*", default=["quantize_bf16", "dequantize_bf16", "gelu_i8", "layernorm_i8"])
+    p.add_argument("--sweep-ops", nargs="*", default=["quantize_bf16", "dequantize_bf16", "gelu_i8", "layernorm_i8",
+                                                      "gelu_i8_bwd", "layernorm_i8_bwd", "fused_fc1"])
     return p.parse_args()
+
+
+ALU_LANES_PER_CLK_PER_SM = 128   # 4 warp schedulers x 32 lanes, one issue per scheduler per clock
+B200_SMS = 148
 
 
 def load_peaks():
@@ -60,7 +65,9 @@ def load_peaks():
     try:
         with open(path) as f:
             d = json.load(f)
-        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+        if any(k not in d for k in ("hbm_gbs", "bf16_tflops")):
+            raise KeyError("incomplete peaks file")
+        return {**FALLBACK_PEAKS, **{k: float(d[k]) for k in FALLBACK_PEAKS if k in d}}, "measured"
     except Exception:
         return dict(FALLBACK_PEAKS), "fallback"
 
@@ -288,11 +295,22 @@ def run_ours(args):
     dom_ms = statistics.mean(per_op[dom])
     achieved = step.ops[dom] / (dom_ms * 1e-3) / 1e12
     traffic = _load_traffic(dom)
-    roofline = {"kernel": f"gemm_i8_kernel ({dom})", "bound": "tensor", "achieved": round(achieved, 1),
-                "peak": round(i8_peak_burst, 1), "unit": "TOPS", "frac": round(achieved / i8_peak_burst, 4),
+    # The binding roofline of the block-scaled GEMM is the SM issue rate, not the tensor pipe: every
+    # output element needs, per 32-deep contraction block, an int32 -> fp32 convert and an FMA (two
+    # lane-instructions), i.e. M*N*K/16 per launch, and an SM issues at most 4 x 32 lane-instructions
+    # per clock. That ceiling (about 1.19 int8 POPS at 1965 MHz) lies below the tensor peak.
+    alu_work = step.ops[dom] // 32                      # 2*M*N*K / 32 = 2 instructions per (element, block)
+    alu_peak = ALU_LANES_PER_CLK_PER_SM * peaks.get("sm_count", B200_SMS) * peaks["sm_max_mhz"] * 1e6 / 1e12
+    alu_achieved = alu_work / (dom_ms * 1e-3) / 1e12
+    roofline = {"kernel": f"gemm_i8_kernel ({dom})", "bound": "alu", "achieved": round(alu_achieved, 2),
+                "peak": round(alu_peak, 2), "unit": "T lane-instructions/s", "frac": round(alu_achieved / alu_peak, 4),
                 "traffic": traffic,
-                "peak_source": f"{peak_src} bf16 dense burst x {NOMINAL_I8_OVER_BF16:g} (nominal int8/bf16 ratio)",
-                "algorithmic": f"2*M*N*K = {step.ops[dom]} int8 ops per launch"}
+                "peak_source": f"{ALU_LANES_PER_CLK_PER_SM} lane-instructions/clk/SM (4 schedulers x 32 lanes) x "
+                               f"{B200_SMS} SMs x {peaks['sm_max_mhz']:g} MHz",
+                "algorithmic": f"2 per output element per 32-deep block = M*N*K/16 = {alu_work} per launch",
+                "tensor_view": {"achieved": round(achieved, 1), "peak": round(i8_peak_burst, 1), "unit": "TOPS",
+                                "frac": round(achieved / i8_peak_burst, 4),
+                                "peak_source": f"{peak_src} bf16 dense burst x {NOMINAL_I8_OVER_BF16:g}"}}
 
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
@@ -319,13 +337,13 @@ def run_ours(args):
 
 def _load_traffic(kernel_op):
     """DRAM read + write bytes per launch of the dominant kernel from the committed ncu capture
-    (profiles/gemm_traffic.json), or None when that capture was taken of other kernel sources."""
+    (profiles/gemm_traffic.json), or None when that capture was taken of other GEMM kernel sources."""
     path = os.path.join(ROOT, "profiles", "gemm_traffic.json")
     try:
         from int8_fully_quantized_b200 import build_lib
         with open(path) as f:
             d = json.load(f)
-        if d.get("source_hash") != build_lib.source_hash():
+        if d.get("kernel_source_hash") != build_lib.kernel_source_hash():
             return None
         v = d.get(kernel_op)
         return None if v is None else int(v)
@@ -453,10 +471,12 @@ def run_reference(args):
 
 
 def run_sweep(args):
-    """Memory-bound sweep: quantize (bf16 in), dequantize (bf16 out), GELU_i8 and LayerNorm_i8 on
-    M x 4096 tensors, M in {1024, 8192, 65536}; N(0,1) with 1% of the channels x100. One JSON line
-    with GB/s (algorithmic bytes: read once, write once) and the fraction of the measured HBM copy
-    bandwidth per kernel and size."""
+    """Memory-bound sweep: quantize (bf16 in), dequantize (bf16 out), GELU_i8, LayerNorm_i8 and their
+    INT8 backward on M x 4096 tensors, M in {1024, 8192, 65536}; N(0,1) with 1% of the channels x100.
+    One JSON line with GB/s (algorithmic bytes: every input read once, every output written once)
+    and the fraction of the measured HBM copy bandwidth per kernel and size. With "fused_fc1" it
+    also times the GPT2-medium fc1 forward with GELU fused into the GEMM epilogue against the
+    forward GEMM followed by GELU_i8."""
     import torch
     import int8_fully_quantized_b200 as jf
     from inputs import synthetic as S
@@ -471,6 +491,8 @@ def run_sweep(args):
         xb = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
         del x
         Q = jf.quantize_block(xb)
+        D = jf.quantize_block(torch.from_numpy(S.to_bf16_bits(S.memory_sweep_input(1, M, H)).view(np.int16)).cuda()
+                              .view(torch.bfloat16))
         Y = jf.empty_qtensor(M, H)
         yb = torch.empty((M, H), dtype=torch.bfloat16, device="cuda")
         gamma = torch.ones(H, device="cuda")
@@ -480,7 +502,12 @@ def run_sweep(args):
             "dequantize_bf16": (lambda: jf.jf_dequantize_block(Q.q, Q.s, yb), M * H * 3 + (M // 32) * (H // 32) * 4),
             "gelu_i8": (lambda: jf.jf_gelu_i8(Q, Y), bytes_i8_op(M, H)),
             "layernorm_i8": (lambda: jf.jf_layernorm_i8(Q, gamma, beta, 1e-5, Y), bytes_i8_op(M, H, 8 * H)),
+            "gelu_i8_bwd": (lambda: jf.jf_gelu_i8_bwd(Q, D, Y), bytes_i8_op(M, H, M * H + (M // 32) * (H // 32) * 4)),
+            "layernorm_i8_bwd": (lambda: jf.jf_layernorm_i8_bwd(Q, D, gamma, 1e-5, Y, dgam, dbet, ws),
+                                 bytes_i8_op(M, H, M * H + (M // 32) * (H // 32) * 4 + 12 * H)),
         }
+        dgam, dbet = torch.empty(H, device="cuda"), torch.empty(H, device="cuda")
+        ws = torch.empty(jf.jf_layernorm_i8_bwd_workspace_bytes(M, H), dtype=torch.uint8, device="cuda")
         for name, (fn, nbytes) in ops.items():
             if name not in args.sweep_ops:
                 continue
@@ -497,10 +524,44 @@ def run_sweep(args):
             ms = statistics.median(a.elapsed_time(b) for a, b in ts)
             gbs = nbytes / (ms * 1e-3) / 1e9
             out[f"{name}@M={M}"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
-        del xb, Q, Y, yb
+        del xb, Q, D, Y, yb, ws
+    if "fused_fc1" in args.sweep_ops:
+        out.update(_sweep_fused_fc1(jf, flush))
     assert jf.jf_device_status() == 0
     print(json.dumps({"sweep": out, "hbm_peak_gbs": peaks["hbm_gbs"], "peak_source": peak_src,
                       "l2": "flushed before every timed launch"}), flush=True)
+
+
+def _sweep_fused_fc1(jf, flush):
+    """GPT2-medium fc1 forward (M=4096, K=1024, N=4096): GELU fused into the GEMM epilogue versus the
+    forward GEMM followed by GELU_i8 (device time of each variant, L2 flushed before each)."""
+    import torch
+    wl = __import__("inputs.synthetic", fromlist=["WORKLOADS"]).WORKLOADS[WORKLOAD]
+    M, K, N = wl["M"], wl["K"], wl["N"]
+    host = host_inputs(M, K, N, 0, seed_weight=0)
+    X = jf.quantize_block(torch.from_numpy(host["x"].view(np.int16)).cuda().view(torch.bfloat16))
+    W = jf.quantize_block(torch.from_numpy(host["w"].view(np.int16)).cuda().view(torch.bfloat16))
+    Y, G, P = jf.empty_qtensor(M, N), jf.empty_qtensor(M, N), jf.empty_qtensor(M, N)
+    variants = {
+        "fc1_fwd_then_gelu_i8": lambda: (jf.jf_linear_fwd(X, W, Y), jf.jf_gelu_i8(Y, G)),
+        "fc1_fwd_gelu_fused": lambda: jf.jf_linear_fwd_gelu(X, W, G),
+        "fc1_fwd_gelu_fused_with_pre": lambda: jf.jf_linear_fwd_gelu(X, W, G, P),
+    }
+    res = {}
+    for name, fn in variants.items():
+        for _ in range(3):
+            flush.zero_()
+            fn()
+        ts = []
+        for _ in range(10):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(); fn(); b.record()
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        ms = statistics.median(a.elapsed_time(b) for a, b in ts)
+        res[name] = {"ms": round(ms, 4), "TOPS": round(2 * M * N * K / (ms * 1e-3) / 1e12, 1)}
+    return res
 
 
 def main():

@@ -173,17 +173,18 @@ JF_API int jf_gelu_i8_bwd(jf_cqtensor X, jf_cqtensor dY, jf_qtensor dX, void* st
  *          and over all rows dgamma = sum dy xhat, dbeta = sum dy (fp32 [H], deterministic).
  *   dgamma, dbeta  nullable device fp32 [H]; when either is given, `workspace` must hold at least
  *          jf_layernorm_i8_bwd_workspace_bytes(M, H) bytes of caller-owned device memory, 16-byte
- *          aligned (per-strip column sums; its contents on entry do not matter). Otherwise the
+ *          aligned (per-CTA column sums; its contents on entry do not matter). Otherwise the
  *          workspace is not used and may be NULL.
- *   Errors: JF_ERR_NULL if gamma or dX.q is NULL; JF_ERR_WORKSPACE as above; JF_ERR_ALIAS if any
- *          output (workspace included) overlaps an input or another output.
+ *   H is at most 24576 (the column sums of a CTA live in shared memory).
+ *   Errors: JF_ERR_NULL if gamma or dX.q is NULL; JF_ERR_SHAPE for H > 24576; JF_ERR_WORKSPACE as
+ *          above; JF_ERR_ALIAS if any output (workspace included) overlaps an input or another output.
  */
 JF_API int jf_layernorm_i8_bwd(jf_cqtensor X, jf_cqtensor dY, const float* gamma, float eps, jf_qtensor dX,
                                float* dgamma, float* dbeta, void* workspace, int64_t workspace_bytes,
                                void* stream);
 
-/* Bytes of workspace jf_layernorm_i8_bwd needs for X of [rows, cols]: (rows / 32) * 2 * cols * 4,
- * or -1 for an invalid shape. */
+/* Bytes of workspace jf_layernorm_i8_bwd needs for X of [rows, cols]:
+ * min(rows / 32, 444) * 2 * cols * 4, or -1 for an invalid shape (cols > 24576 included). */
 JF_API int64_t jf_layernorm_i8_bwd_workspace_bytes(int64_t rows, int64_t cols);
 
 /* Static description of a status code (never NULL). */

@@ -51,6 +51,21 @@ def source_hash() -> str:
     return h.hexdigest()
 
 
+# Files that define the block-scaled GEMM kernel's device code (its host launcher lives in gemm.cu too).
+GEMM_KERNEL_FILES = ("gemm.cu", "ptx.cuh", "quant.cuh", "act.cuh")
+
+
+def kernel_source_hash(names=GEMM_KERNEL_FILES) -> str:
+    """Content hash of the given csrc files only: a record taken of one kernel (e.g. its ncu DRAM
+    traffic) stays valid while these files are unchanged, whatever else in the library changes."""
+    h = hashlib.sha256()
+    for n in sorted(names):
+        h.update(n.encode())
+        with open(os.path.join(CSRC, n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def built_hash() -> str | None:
     try:
         with open(HASH_PATH) as f:

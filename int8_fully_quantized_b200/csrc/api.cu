@@ -264,8 +264,8 @@ int jf_gelu_i8_bwd(jf_cqtensor X, jf_cqtensor dY, jf_qtensor dX, void* stream) {
 }
 
 int64_t jf_layernorm_i8_bwd_workspace_bytes(int64_t rows, int64_t cols) {
-  if (!dims_ok(rows, cols)) return -1;
-  return (rows / 32) * 2 * cols * 4;
+  if (!dims_ok(rows, cols) || cols > jf::kLnBwdMaxCols) return -1;
+  return jf::ln_bwd_ctas(rows) * 2 * cols * 4;
 }
 
 int jf_layernorm_i8_bwd(jf_cqtensor X, jf_cqtensor dY, const float* gamma, float eps, jf_qtensor dX, float* dgamma,
@@ -275,6 +275,7 @@ int jf_layernorm_i8_bwd(jf_cqtensor X, jf_cqtensor dY, const float* gamma, float
   if ((st = check_cq(dY)) != JF_OK) return st;
   if ((st = check_q(dX, true)) != JF_OK) return st;
   if (X.rows != dY.rows || X.cols != dY.cols || X.rows != dX.rows || X.cols != dX.cols) return JF_ERR_SHAPE;
+  if (X.cols > jf::kLnBwdMaxCols) return JF_ERR_SHAPE;
   if (X.rows == 0 || X.cols == 0) return JF_OK;
   if (gamma == nullptr) return JF_ERR_NULL;
   if (!aligned(gamma, 16) || !aligned(dgamma, 4) || !aligned(dbeta, 4)) return JF_ERR_ALIGN;

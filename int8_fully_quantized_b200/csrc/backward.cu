@@ -76,160 +76,176 @@ __global__ void __launch_bounds__(32 * kGeluBwdWarps, 3) gelu_i8_bwd_kernel(
 // LayerNorm_i8 backward. For the layer y = (x - mu) rstd gamma + beta (mu, biased variance over the
 // H columns of a row, rstd = 1 / sqrt(var + eps)), with xhat = (x - mu) rstd and g = dy gamma:
 //   dx = rstd (g - mean(g) - xhat mean(g xhat)),  dgamma = sum_rows dy xhat,  dbeta = sum_rows dy.
-// One CTA of 8 warps per 32-row strip, three CTAs per SM:
-//   phase 1: warp w reduces rows w, w + 8, w + 16 and w + 24, each in one pass: sums of x, x^2, g and g x (chunk partials
+// Persistent CTAs of 8 warps, three per SM, each looping over 32-row strips:
+//   phase 1: warp w reduces rows w, w + 8, w + 16 and w + 24 of the strip, each in one pass: sums of x, x^2, g and g x (chunk partials
 //            of 16 values in fp32, accumulated in fp64). Then mean, rstd, mean(g) and
 //            mean(g xhat) = rstd (mean(g x) - mean * mean(g)) per row, kept in shared memory.
 //   phase 2: warp w handles column blocks w, w + 8, ...: lane l takes the 4 columns 4 (l % 8) .. +3
 //            of rows l / 8 + 4 i (i = 0..7), computes dx, re-quantizes the block and sums dy xhat
 //            and dy of its columns over the strip's 32 rows (shuffles across the 4 row groups).
 //            The strip (2 x 32 H bytes) is read a second time, from L2.
-//   The per-strip column sums go to part[strip][0 | 1][H] when gamma or beta gradients are asked
-//   for; ln_bwd_reduce_kernel then adds them over the strips in a fixed order (deterministic).
+//   When gamma or beta gradients are asked for, a CTA adds each strip's column sums into fp32
+//   accumulators in shared memory (every column belongs to one warp, so no atomics), writes them
+//   to part[cta][0 | 1][H] at the end, and ln_bwd_reduce_kernel adds the CTAs' partials in a fixed
+//   order. The workspace is ln_bwd_ctas(R) * 2 * H floats, independent of R beyond 444 strips.
 // ---------------------------------------------------------------------------------------------
 constexpr int kLnbThreads = 256;
+
+int64_t ln_bwd_ctas(int64_t R) { return R / 32 < kLnBwdMaxCtas ? R / 32 : kLnBwdMaxCtas; }
 
 __global__ void __launch_bounds__(kLnbThreads, 3) layernorm_i8_bwd_kernel(
     const int8_t* __restrict__ xq, const float* __restrict__ xs, const int8_t* __restrict__ dq,
     const float* __restrict__ ds, int64_t R, int64_t H, const float* __restrict__ gamma, float eps,
     int8_t* __restrict__ qo, float* __restrict__ so, float* __restrict__ part) {
   __shared__ float4 s_stat[32];  // per row: mean, rstd, mean(g), mean(g xhat)
+  extern __shared__ float s_acc[];  // [2][H] column sums of dy xhat and dy over this CTA's strips
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t strip = blockIdx.x;
   const int64_t nbc = H >> 5;
-  const int8_t* xstrip = xq + strip * 32 * H;
-  const int8_t* dstrip = dq + strip * 32 * H;
-  const float* xss = xs + strip * nbc;
-  const float* dss = ds + strip * nbc;
-  for (int rw = warp; rw < 32; rw += kLnbThreads / 32) {
-    const int8_t* xrow = xstrip + int64_t(rw) * H;
-    const int8_t* drow = dstrip + int64_t(rw) * H;
-    double sum_x = 0.0, sum_xx = 0.0, sum_g = 0.0, sum_gx = 0.0;
-    constexpr int kUnroll = 4;  // 16-byte chunks of each tensor a lane keeps in flight
-    for (int64_t ch0 = lane; ch0 < (H >> 4); ch0 += 32 * kUnroll) {
-      uint4 av[kUnroll], dv[kUnroll];
-      float scx[kUnroll], scd[kUnroll];
+  if (part != nullptr)
+    for (int64_t c = threadIdx.x; c < 2 * H; c += kLnbThreads) s_acc[c] = 0.0f;
+  for (int64_t strip = blockIdx.x; strip < (R >> 5); strip += gridDim.x) {
+    __syncthreads();  // s_stat is rewritten for this strip only after every warp has used the last one
+    const int8_t* xstrip = xq + strip * 32 * H;
+    const int8_t* dstrip = dq + strip * 32 * H;
+    const float* xss = xs + strip * nbc;
+    const float* dss = ds + strip * nbc;
+    for (int rw = warp; rw < 32; rw += kLnbThreads / 32) {
+      const int8_t* xrow = xstrip + int64_t(rw) * H;
+      const int8_t* drow = dstrip + int64_t(rw) * H;
+      double sum_x = 0.0, sum_xx = 0.0, sum_g = 0.0, sum_gx = 0.0;
+      constexpr int kUnroll = 4;  // 16-byte chunks of each tensor a lane keeps in flight
+      for (int64_t ch0 = lane; ch0 < (H >> 4); ch0 += 32 * kUnroll) {
+        uint4 av[kUnroll], dv[kUnroll];
+        float scx[kUnroll], scd[kUnroll];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int64_t ch = ch0 + 32 * u;
-        if (ch < (H >> 4)) {
-          av[u] = ld_stream_v4(xrow + ch * 16);
-          dv[u] = ld_stream_v4(drow + ch * 16);
-          scx[u] = __ldg(xss + (ch >> 1));
-          scd[u] = __ldg(dss + (ch >> 1));
-        } else {
-          av[u] = dv[u] = make_uint4(0u, 0u, 0u, 0u);
-          scx[u] = scd[u] = 0.0f;
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int64_t ch = ch0 + 32 * u;
-        if (ch >= (H >> 4)) break;
-        const uint32_t wx[4] = {av[u].x, av[u].y, av[u].z, av[u].w};
-        const uint32_t wd[4] = {dv[u].x, dv[u].y, dv[u].z, dv[u].w};
-        const float4* g4 = reinterpret_cast<const float4*>(gamma + ch * 16);
-        float px = 0.0f, pxx = 0.0f, pg = 0.0f, pgx = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float4 gm = __ldg(g4 + i);
-          const float gmv[4] = {gm.x, gm.y, gm.z, gm.w};
-          float fx[4], fd[4];
-          i8x4_to_f32(wx[i], fx);
-          i8x4_to_f32(wd[i], fd);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float x = fx[j] * scx[u];
-            const float g = (fd[j] * scd[u]) * gmv[j];
-            px += x;
-            pxx = fmaf(x, x, pxx);
-            pg += g;
-            pgx = fmaf(g, x, pgx);
+        for (int u = 0; u < kUnroll; ++u) {
+          const int64_t ch = ch0 + 32 * u;
+          if (ch < (H >> 4)) {
+            av[u] = ld_stream_v4(xrow + ch * 16);
+            dv[u] = ld_stream_v4(drow + ch * 16);
+            scx[u] = __ldg(xss + (ch >> 1));
+            scd[u] = __ldg(dss + (ch >> 1));
+          } else {
+            av[u] = dv[u] = make_uint4(0u, 0u, 0u, 0u);
+            scx[u] = scd[u] = 0.0f;
           }
         }
-        sum_x += double(px);
-        sum_xx += double(pxx);
-        sum_g += double(pg);
-        sum_gx += double(pgx);
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const int64_t ch = ch0 + 32 * u;
+          if (ch >= (H >> 4)) break;
+          const uint32_t wx[4] = {av[u].x, av[u].y, av[u].z, av[u].w};
+          const uint32_t wd[4] = {dv[u].x, dv[u].y, dv[u].z, dv[u].w};
+          const float4* g4 = reinterpret_cast<const float4*>(gamma + ch * 16);
+          float px = 0.0f, pxx = 0.0f, pg = 0.0f, pgx = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float4 gm = __ldg(g4 + i);
+            const float gmv[4] = {gm.x, gm.y, gm.z, gm.w};
+            float fx[4], fd[4];
+            i8x4_to_f32(wx[i], fx);
+            i8x4_to_f32(wd[i], fd);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float x = fx[j] * scx[u];
+              const float g = (fd[j] * scd[u]) * gmv[j];
+              px += x;
+              pxx = fmaf(x, x, pxx);
+              pg += g;
+              pgx = fmaf(g, x, pgx);
+            }
+          }
+          sum_x += double(px);
+          sum_xx += double(pxx);
+          sum_g += double(pg);
+          sum_gx += double(pgx);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        sum_x += __shfl_xor_sync(0xffffffffu, sum_x, o);
+        sum_xx += __shfl_xor_sync(0xffffffffu, sum_xx, o);
+        sum_g += __shfl_xor_sync(0xffffffffu, sum_g, o);
+        sum_gx += __shfl_xor_sync(0xffffffffu, sum_gx, o);
+      }
+      if (lane == 0) {
+        const double inv_h = 1.0 / double(H);
+        const double mean = sum_x * inv_h;
+        double var = sum_xx * inv_h - mean * mean;
+        var = var > 0.0 ? var : 0.0;
+        const double rstd = 1.0 / sqrt(var + double(eps));
+        const double mg = sum_g * inv_h;
+        const double mgx = rstd * (sum_gx * inv_h - mean * mg);
+        s_stat[rw] = make_float4(float(mean), float(rstd), float(mg), float(mgx));
       }
     }
+    __syncthreads();
+    const int cg = lane & 7, rg = lane >> 3;
+    for (int64_t bj = warp; bj < nbc; bj += kLnbThreads / 32) {
+      const float sx = __ldg(xss + bj), sd = __ldg(dss + bj);
+      const int64_t col = bj * 32 + 4 * cg;
+      const float4 gm4 = __ldg(reinterpret_cast<const float4*>(gamma + col));
+      const float gm[4] = {gm4.x, gm4.y, gm4.z, gm4.w};
+      uint32_t wx[8], wd[8];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      sum_x += __shfl_xor_sync(0xffffffffu, sum_x, o);
-      sum_xx += __shfl_xor_sync(0xffffffffu, sum_xx, o);
-      sum_g += __shfl_xor_sync(0xffffffffu, sum_g, o);
-      sum_gx += __shfl_xor_sync(0xffffffffu, sum_gx, o);
-    }
-    if (lane == 0) {
-      const double inv_h = 1.0 / double(H);
-      const double mean = sum_x * inv_h;
-      double var = sum_xx * inv_h - mean * mean;
-      var = var > 0.0 ? var : 0.0;
-      const double rstd = 1.0 / sqrt(var + double(eps));
-      const double mg = sum_g * inv_h;
-      const double mgx = rstd * (sum_gx * inv_h - mean * mg);
-      s_stat[rw] = make_float4(float(mean), float(rstd), float(mg), float(mgx));
+      for (int i = 0; i < 8; ++i) {
+        const int64_t off = int64_t(rg + 4 * i) * H + col;
+        wx[i] = ld_stream_b32(xstrip + off);
+        wd[i] = ld_stream_b32(dstrip + off);
+      }
+      float v[32], pgam[4] = {0.0f, 0.0f, 0.0f, 0.0f}, pbet[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      float m = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float fx[4], fd[4];
+        i8x4_to_f32(wx[i], fx);
+        i8x4_to_f32(wd[i], fd);
+        const float4 st = s_stat[rg + 4 * i];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float xhat = (fx[j] * sx - st.x) * st.y;
+          const float dy = fd[j] * sd;
+          const float dx = st.y * (fmaf(dy, gm[j], -st.z) - xhat * st.w);
+          v[4 * i + j] = dx;
+          m = fmaxf(m, fabsf(dx));
+          pgam[j] = fmaf(dy, xhat, pgam[j]);
+          pbet[j] += dy;
+        }
+      }
+      const BlockQuant bq = block_quant(warp_max_nonneg(m));
+      uint32_t o[8];
+      quant_pack<32>(v, bq, o);
+      int8_t* dst = qo + strip * 32 * H;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) *reinterpret_cast<uint32_t*>(dst + int64_t(rg + 4 * i) * H + col) = o[i];
+      if (lane == 0) so[strip * nbc + bj] = bq.s;
+      if (part != nullptr) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          pgam[j] += __shfl_xor_sync(0xffffffffu, pgam[j], 8);
+          pgam[j] += __shfl_xor_sync(0xffffffffu, pgam[j], 16);
+          pbet[j] += __shfl_xor_sync(0xffffffffu, pbet[j], 8);
+          pbet[j] += __shfl_xor_sync(0xffffffffu, pbet[j], 16);
+        }
+        if (rg == 0) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            s_acc[col + j] += pgam[j];
+            s_acc[H + col + j] += pbet[j];
+          }
+        }
+      }
     }
   }
-  __syncthreads();
-  const int cg = lane & 7, rg = lane >> 3;
-  for (int64_t bj = warp; bj < nbc; bj += kLnbThreads / 32) {
-    const float sx = __ldg(xss + bj), sd = __ldg(dss + bj);
-    const int64_t col = bj * 32 + 4 * cg;
-    const float4 gm4 = __ldg(reinterpret_cast<const float4*>(gamma + col));
-    const float gm[4] = {gm4.x, gm4.y, gm4.z, gm4.w};
-    uint32_t wx[8], wd[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int64_t off = int64_t(rg + 4 * i) * H + col;
-      wx[i] = ld_stream_b32(xstrip + off);
-      wd[i] = ld_stream_b32(dstrip + off);
-    }
-    float v[32], pgam[4] = {0.0f, 0.0f, 0.0f, 0.0f}, pbet[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    float m = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float fx[4], fd[4];
-      i8x4_to_f32(wx[i], fx);
-      i8x4_to_f32(wd[i], fd);
-      const float4 st = s_stat[rg + 4 * i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float xhat = (fx[j] * sx - st.x) * st.y;
-        const float dy = fd[j] * sd;
-        const float dx = st.y * (fmaf(dy, gm[j], -st.z) - xhat * st.w);
-        v[4 * i + j] = dx;
-        m = fmaxf(m, fabsf(dx));
-        pgam[j] = fmaf(dy, xhat, pgam[j]);
-        pbet[j] += dy;
-      }
-    }
-    const BlockQuant bq = block_quant(warp_max_nonneg(m));
-    uint32_t o[8];
-    quant_pack<32>(v, bq, o);
-    int8_t* dst = qo + strip * 32 * H;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) *reinterpret_cast<uint32_t*>(dst + int64_t(rg + 4 * i) * H + col) = o[i];
-    if (lane == 0) so[strip * nbc + bj] = bq.s;
-    if (part != nullptr) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        pgam[j] += __shfl_xor_sync(0xffffffffu, pgam[j], 8);
-        pgam[j] += __shfl_xor_sync(0xffffffffu, pgam[j], 16);
-        pbet[j] += __shfl_xor_sync(0xffffffffu, pbet[j], 8);
-        pbet[j] += __shfl_xor_sync(0xffffffffu, pbet[j], 16);
-      }
-      if (rg == 0) {
-        float* pg = part + strip * 2 * H;
-        *reinterpret_cast<float4*>(pg + col) = make_float4(pgam[0], pgam[1], pgam[2], pgam[3]);
-        *reinterpret_cast<float4*>(pg + H + col) = make_float4(pbet[0], pbet[1], pbet[2], pbet[3]);
-      }
-    }
+  if (part != nullptr) {
+    __syncthreads();
+    float* pg = part + int64_t(blockIdx.x) * 2 * H;
+    for (int64_t c = threadIdx.x; c < 2 * H; c += kLnbThreads) pg[c] = s_acc[c];
   }
 }
 
-// dgamma[c] and dbeta[c] = sums over the strips of part[strip][0 | 1][c], in fp64 and in a fixed
-// order (warp w adds strips w, w + 8, ...; the 8 warp sums are then added in warp order), so the
+// dgamma[c] and dbeta[c] = sums over the CTAs' partials part[k][0 | 1][c], in fp64 and in a fixed
+// order (warp w adds partials w, w + 8, ...; the 8 warp sums are then added in warp order), so the
 // result does not depend on scheduling. One CTA per 32 columns, lane = column.
 __global__ void __launch_bounds__(256) ln_bwd_reduce_kernel(const float* __restrict__ part, int64_t nstrips,
                                                             int64_t H, float* __restrict__ dgamma,
@@ -273,10 +289,18 @@ cudaError_t launch_gelu_i8_bwd(const int8_t* xq, const float* xs, const int8_t* 
 cudaError_t launch_layernorm_i8_bwd(const int8_t* xq, const float* xs, const int8_t* dq, const float* ds, int64_t R,
                                     int64_t H, const float* gamma, float eps, int8_t* qo, float* so, float* part,
                                     float* dgamma, float* dbeta, cudaStream_t st) {
-  layernorm_i8_bwd_kernel<<<int(R / 32), kLnbThreads, 0, st>>>(xq, xs, dq, ds, R, H, gamma, eps, qo, so, part);
+  // persistent CTAs only when they accumulate column sums; otherwise one CTA per strip
+  const int grid = int(part != nullptr ? ln_bwd_ctas(R) : R / 32);
+  const size_t smem = part != nullptr ? size_t(H) * 2 * sizeof(float) : 0;
+  if (smem > 48 * 1024) {
+    const cudaError_t a = cudaFuncSetAttribute(layernorm_i8_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               int(smem));
+    if (a != cudaSuccess) return a;
+  }
+  layernorm_i8_bwd_kernel<<<grid, kLnbThreads, smem, st>>>(xq, xs, dq, ds, R, H, gamma, eps, qo, so, part);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || part == nullptr) return e;
-  ln_bwd_reduce_kernel<<<int(H / 32), 256, 0, st>>>(part, R / 32, H, dgamma, dbeta);
+  ln_bwd_reduce_kernel<<<int(H / 32), 256, 0, st>>>(part, grid, H, dgamma, dbeta);
   return cudaGetLastError();
 }
 

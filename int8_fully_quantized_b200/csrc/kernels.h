@@ -12,8 +12,11 @@ cudaError_t launch_dequantize(const int8_t* q, const float* s, int64_t R, int64_
                               int sm_count, cudaStream_t st);
 cudaError_t launch_gelu_i8(const int8_t* q, const float* s, int64_t R, int64_t C, int8_t* qo, float* so,
                            int sm_count, cudaStream_t st);
-// INT8 backward of GELU_i8 and LayerNorm_i8 (backward.cu). `part` is the [R/32][2][H] fp32
-// workspace of per-strip column sums; null when neither dgamma nor dbeta is wanted.
+// INT8 backward of GELU_i8 and LayerNorm_i8 (backward.cu). `part` is the fp32 workspace of
+// per-CTA column sums, [ln_bwd_ctas(R)][2][H]; null when neither dgamma nor dbeta is wanted.
+constexpr int64_t kLnBwdMaxCtas = 444;   // three resident CTAs on each of 148 SMs
+constexpr int64_t kLnBwdMaxCols = 24576; // the [2][H] fp32 accumulators fit in one SM's shared memory
+int64_t ln_bwd_ctas(int64_t R);
 cudaError_t launch_gelu_i8_bwd(const int8_t* xq, const float* xs, const int8_t* dq, const float* ds, int64_t R,
                                int64_t C, int8_t* qo, float* so, int sm_count, cudaStream_t st);
 cudaError_t launch_layernorm_i8_bwd(const int8_t* xq, const float* xs, const int8_t* dq, const float* ds, int64_t R,
