@@ -187,6 +187,19 @@ JF_API int jf_layernorm_i8_bwd(jf_cqtensor X, jf_cqtensor dY, const float* gamma
  * min(rows / 32, 444) * 2 * cols * 4, or -1 for an invalid shape (cols > 24576 included). */
 JF_API int64_t jf_layernorm_i8_bwd_workspace_bytes(int64_t rows, int64_t cols);
 
+/*
+ * Allocation-free variant of jf_layernorm_i8_bwd (no counterpart on the pages: an engineering entry
+ * point for callers that cannot provide a workspace). Same arguments, results and errors, but the
+ * per-CTA column sums go to a 16 MiB scratch array that the library holds in device memory for
+ * its whole lifetime, so neither the caller nor the library allocates anything per call. Shapes
+ * whose workspace (jf_layernorm_i8_bwd_workspace_bytes) exceeds 16 MiB are rejected with
+ * JF_ERR_WORKSPACE before anything is enqueued. The scratch is shared by every call on a device:
+ * calls of this function that ask for dgamma or dbeta must not run concurrently with each other
+ * (issue them on one stream). Without dgamma and dbeta it is jf_layernorm_i8_bwd with no workspace.
+ */
+JF_API int jf_layernorm_i8_bwd_noalloc(jf_cqtensor X, jf_cqtensor dY, const float* gamma, float eps,
+                                       jf_qtensor dX, float* dgamma, float* dbeta, void* stream);
+
 /* Static description of a status code (never NULL). */
 JF_API const char* jf_strerror(int status);
 

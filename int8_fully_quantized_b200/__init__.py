@@ -24,7 +24,8 @@ from .build_lib import LIB_PATH
 __all__ = [
     "QTensor", "JetfireError", "load_library", "empty_qtensor", "jf_quantize_block", "jf_dequantize_block",
     "jf_linear_fwd", "jf_linear_fwd_gelu", "jf_linear_dgrad", "jf_linear_wgrad", "jf_gelu_i8", "jf_layernorm_i8",
-    "jf_gelu_i8_bwd", "jf_layernorm_i8_bwd", "jf_layernorm_i8_bwd_workspace_bytes", "gelu_i8_bwd",
+    "jf_gelu_i8_bwd", "jf_layernorm_i8_bwd", "jf_layernorm_i8_bwd_workspace_bytes", "jf_layernorm_i8_bwd_noalloc",
+    "gelu_i8_bwd",
     "layernorm_i8_bwd", "jf_strerror", "jf_device_status", "jf_sm_count", "quantize_block", "dequantize_block",
     "linear_fwd",
     "linear_fwd_gelu", "linear_dgrad",
@@ -38,6 +39,7 @@ EXPORTED_SYMBOLS = (
     "jf_quantize_block", "jf_dequantize_block", "jf_linear_fwd", "jf_linear_fwd_gelu", "jf_linear_dgrad",
     "jf_linear_wgrad",
     "jf_gelu_i8", "jf_layernorm_i8", "jf_gelu_i8_bwd", "jf_layernorm_i8_bwd", "jf_layernorm_i8_bwd_workspace_bytes",
+    "jf_layernorm_i8_bwd_noalloc",
     "jf_strerror", "jf_device_status", "jf_sm_count",
 )
 
@@ -82,6 +84,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.jf_gelu_i8_bwd.argtypes = [_CQ, _CQ, _Q, vp]
     lib.jf_layernorm_i8_bwd.argtypes = [_CQ, _CQ, vp, ctypes.c_float, _Q, vp, vp, vp, i64, vp]
     lib.jf_layernorm_i8_bwd_workspace_bytes.argtypes = [i64, i64]
+    lib.jf_layernorm_i8_bwd_noalloc.argtypes = [_CQ, _CQ, vp, ctypes.c_float, _Q, vp, vp, vp]
     lib.jf_strerror.argtypes = [i32]
     lib.jf_strerror.restype = ctypes.c_char_p
     lib.jf_device_status.argtypes = [vp]
@@ -213,6 +216,14 @@ def jf_layernorm_i8_bwd(X: QTensor, dY: QTensor, gamma: torch.Tensor, eps: float
     _check(lib.jf_layernorm_i8_bwd(_cq(X), _cq(dY), _ptr(gamma), ctypes.c_float(eps), _q(dX, X.rows, X.cols),
                                    _ptr(dgamma), _ptr(dbeta), _ptr(workspace), nbytes, _stream(stream)),
            "jf_layernorm_i8_bwd")
+
+
+def jf_layernorm_i8_bwd_noalloc(X: QTensor, dY: QTensor, gamma: torch.Tensor, eps: float, dX: QTensor,
+                                dgamma: Optional[torch.Tensor] = None, dbeta: Optional[torch.Tensor] = None,
+                                stream=None) -> None:
+    lib = load_library()
+    _check(lib.jf_layernorm_i8_bwd_noalloc(_cq(X), _cq(dY), _ptr(gamma), ctypes.c_float(eps), _q(dX, X.rows, X.cols),
+                                           _ptr(dgamma), _ptr(dbeta), _stream(stream)), "jf_layernorm_i8_bwd_noalloc")
 
 
 def jf_strerror(status: int) -> str:

@@ -303,6 +303,21 @@ int jf_layernorm_i8_bwd(jf_cqtensor X, jf_cqtensor dY, const float* gamma, float
                                                  dgamma, dbeta, static_cast<cudaStream_t>(stream)));
 }
 
+int jf_layernorm_i8_bwd_noalloc(jf_cqtensor X, jf_cqtensor dY, const float* gamma, float eps, jf_qtensor dX,
+                                float* dgamma, float* dbeta, void* stream) {
+  if (dgamma == nullptr && dbeta == nullptr)
+    return jf_layernorm_i8_bwd(X, dY, gamma, eps, dX, nullptr, nullptr, nullptr, 0, stream);
+  const int64_t need = jf_layernorm_i8_bwd_workspace_bytes(X.rows, X.cols);
+  if (need < 0) return JF_ERR_SHAPE;
+  if (need > jf::kLnBwdScratchBytes) return JF_ERR_WORKSPACE;  // larger than the static scratch
+  if (X.rows == 0 || X.cols == 0) return jf_layernorm_i8_bwd(X, dY, gamma, eps, dX, dgamma, dbeta, nullptr, 0, stream);
+  const DevInfo d = device_info();
+  if (!d.ok) return JF_ERR_DEVICE;
+  float* scratch = jf::ln_bwd_static_scratch();
+  if (scratch == nullptr) return JF_ERR_CUDA;
+  return jf_layernorm_i8_bwd(X, dY, gamma, eps, dX, dgamma, dbeta, scratch, jf::kLnBwdScratchBytes, stream);
+}
+
 const char* jf_strerror(int status) {
   switch (status) {
     case JF_OK: return "ok";

@@ -5,6 +5,8 @@
 // pass as in the forward. Both kernels here are memory-bound: they read two INT8 tensors (the
 // saved forward input and the upstream gradient) and write one, re-quantized per block on chip.
 #include <cstdint>
+#include <mutex>
+
 #include <cuda_runtime.h>
 
 #include "act.cuh"
@@ -271,6 +273,27 @@ __global__ void __launch_bounds__(256) ln_bwd_reduce_kernel(const float* __restr
     if (dgamma != nullptr) dgamma[col] = float(tg);
     if (dbeta != nullptr) dbeta[col] = float(tb);
   }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Static scratch of the allocation-free LayerNorm backward: the per-CTA column sums live in this
+// file-scope device array instead of a caller workspace. Its device address is looked up once per
+// device and cached.
+// ---------------------------------------------------------------------------------------------
+static __device__ __align__(256) float g_ln_bwd_scratch[kLnBwdScratchBytes / sizeof(float)];
+
+float* ln_bwd_static_scratch() {
+  static std::mutex mu;
+  static float* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_ln_bwd_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<float*>(p);
+  }
+  return addr[dev];
 }
 
 // ---------------------------------------------------------------------------------------------

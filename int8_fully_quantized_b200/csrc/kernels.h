@@ -17,6 +17,10 @@ cudaError_t launch_gelu_i8(const int8_t* q, const float* s, int64_t R, int64_t C
 constexpr int64_t kLnBwdMaxCtas = 444;   // three resident CTAs on each of 148 SMs
 constexpr int64_t kLnBwdMaxCols = 24576; // the [2][H] fp32 accumulators fit in one SM's shared memory
 int64_t ln_bwd_ctas(int64_t R);
+// Size of the static scratch the allocation-free LayerNorm backward uses in place of a workspace,
+// and its device address on the current device (looked up once per device; null on failure).
+constexpr int64_t kLnBwdScratchBytes = int64_t(16) << 20;
+float* ln_bwd_static_scratch();
 cudaError_t launch_gelu_i8_bwd(const int8_t* xq, const float* xs, const int8_t* dq, const float* ds, int64_t R,
                                int64_t C, int8_t* qo, float* so, int sm_count, cudaStream_t st);
 cudaError_t launch_layernorm_i8_bwd(const int8_t* xq, const float* xs, const int8_t* dq, const float* ds, int64_t R,

@@ -106,6 +106,9 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert lib.jf_layernorm_i8_bwd(Xc, dYc, None, f, dXq, dg, db, ws, need, None) == -1
     assert lib.jf_layernorm_i8_bwd(Xc, dYc, g, f, dXq, dg, vp((1 << 33) + 8), ws, need, None) == -5
     assert lib.jf_layernorm_i8_bwd(Xc, dYc, g, f, dXq, dg, db, vp((1 << 34) + 16), need, None) == -5
+    # the allocation-free backward refuses shapes whose column sums exceed its 16 MiB static scratch
+    big = jf._CQ(1 << 20, 1 << 22, 32768, 8192)
+    assert lib.jf_layernorm_i8_bwd_noalloc(big, big, g, f, jf._Q(1 << 28, 1 << 30, 32768, 8192), dg, db, None) == -9
     # LayerNorm needs gamma/beta
     assert lib.jf_layernorm_i8(jf._CQ(1 << 20, 1 << 22, 32, 64), None, fake, ctypes.c_float(1e-5),
                                jf._Q(1 << 28, 1 << 30, 32, 64), None) == -1
