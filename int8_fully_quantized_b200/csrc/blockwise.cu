@@ -80,60 +80,85 @@ struct Vec<__half> {
 };
 
 // ---------------------------------------------------------------------------------------------
-// a1: quantize. One warp per 32x32 block. A block row of T is VPR 16-byte vectors; lane l reads
-// vector column l % VPR of rows l / VPR + t * (32 / VPR), so each load instruction covers whole
-// block rows (full 32-byte sectors).
+// a1: quantize. One warp per pair of horizontally adjacent 32x32 blocks (a 32 x 64 tile), so that
+// every store instruction writes whole 64-byte segments of the INT8 output rows: a warp that wrote
+// only its block's 32-byte half of a segment would make L2 fetch the other half from DRAM first
+// (measured: the one-block-per-warp kernel read 1.5x its input). A tile row is VPR 16-byte vectors;
+// lane l reads vector column l % VPR of rows l / VPR + t * RSTEP, so each load instruction covers
+// whole tile rows. The lane keeps only the raw vectors: the block absmax comes from the bit
+// patterns (fp32, bf16 and fp16 are sign-magnitude, so |x| orders like the bits with the sign
+// cleared), reduced over the 16 lanes of the lane's block, and the values are unpacked and quantized
+// eight at a time. When the number of block columns is odd the last pair holds one block.
 // ---------------------------------------------------------------------------------------------
 template <typename T>
-__global__ void __launch_bounds__(256, 4) quantize_kernel(const T* __restrict__ x, int64_t R, int64_t C,
+__device__ __forceinline__ float abs_max_of_bits(uint32_t m);  // m: the largest |x| bit pattern
+template <>
+__device__ __forceinline__ float abs_max_of_bits<float>(uint32_t m) { return __uint_as_float(m); }
+template <>
+__device__ __forceinline__ float abs_max_of_bits<__nv_bfloat16>(uint32_t m) { return __uint_as_float(m << 16); }
+template <>
+__device__ __forceinline__ float abs_max_of_bits<__half>(uint32_t m) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(m)));
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256, 3) quantize_kernel(const T* __restrict__ x, int64_t R, int64_t C,
                                                           int8_t* __restrict__ q, float* __restrict__ s) {
   constexpr int EPV = Vec<T>::kElems;      // elements per 16-byte vector
-  constexpr int VPR = 32 / EPV;            // vectors per block row (= vectors per lane)
+  constexpr int VPR = 64 / EPV;            // vectors per tile row (= vectors per lane)
   constexpr int RSTEP = 32 / VPR;          // rows between a lane's vectors
+  constexpr int HALF = VPR / 2;            // vectors per block row
+  constexpr int VPG = 8 / EPV;             // vectors per group of eight values (1 or 2)
   const int lane = threadIdx.x & 31;
   const int64_t nbc = C >> 5;
-  const int64_t nblocks = (R >> 5) * nbc;
+  const int64_t npc = (nbc + 1) >> 1;      // block pairs per block row
+  const int64_t npairs = (R >> 5) * npc;
   const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
   const int r0 = lane / VPR, vc = lane % VPR;
-  auto src_of = [&](int64_t b) {
-    const int64_t bi = b / nbc, bj = b - bi * nbc;
-    return x + (bi * 32 + r0) * C + bj * 32 + vc * EPV;
-  };
-  int64_t b = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  uint4 raw[VPR];
-  if (b < nblocks) {
-    const T* src = src_of(b);
+  const int half = vc / HALF;              // the block of the pair this lane's columns belong to
+  for (int64_t p = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; p < npairs; p += nwarps) {
+    const int64_t bi = p / npc, pj = p - bi * npc;
+    const int64_t bj = 2 * pj + half;
+    const bool active = bj < nbc;
+    const int64_t off = (bi * 32 + r0) * C + pj * 64 + vc * EPV;
+    uint4 raw[VPR];
 #pragma unroll
-    for (int t = 0; t < VPR; ++t) raw[t] = ld_stream_v4(src + int64_t(t) * RSTEP * C);
-  }
-  for (; b < nblocks; b += nwarps) {
-    float v[VPR * EPV];
-#pragma unroll
-    for (int t = 0; t < VPR; ++t) Vec<T>::unpack(raw[t], *reinterpret_cast<float(*)[EPV]>(v + t * EPV));
-    // the next block's loads are in flight while this block is quantized
-    const int64_t bn = b + nwarps;
-    if (bn < nblocks) {
-      const T* src = src_of(bn);
-#pragma unroll
-      for (int t = 0; t < VPR; ++t) raw[t] = ld_stream_v4(src + int64_t(t) * RSTEP * C);
-    }
-    float m = 0.0f;
-#pragma unroll
-    for (int i = 0; i < VPR * EPV; ++i) m = fmaxf(m, fabsf(v[i]));
-    const BlockQuant bq = block_quant(warp_max_nonneg(m));
-    uint32_t w[VPR * EPV / 4];
-    quant_pack<VPR * EPV>(v, bq, w);
-    const int64_t bi = b / nbc, bj = b - bi * nbc;
-    int8_t* dst = q + (bi * 32 + r0) * C + bj * 32 + vc * EPV;
+    for (int t = 0; t < VPR; ++t)
+      raw[t] = active ? ld_stream_v4(x + off + int64_t(t) * RSTEP * C) : make_uint4(0u, 0u, 0u, 0u);
+    // largest |x| bit pattern of the lane's values
+    uint32_t mb = 0;
 #pragma unroll
     for (int t = 0; t < VPR; ++t) {
-      if constexpr (EPV == 4) {
-        *reinterpret_cast<uint32_t*>(dst + int64_t(t) * RSTEP * C) = w[t];
-      } else {
-        *reinterpret_cast<uint2*>(dst + int64_t(t) * RSTEP * C) = make_uint2(w[2 * t], w[2 * t + 1]);
+      const uint32_t w[4] = {raw[t].x, raw[t].y, raw[t].z, raw[t].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if constexpr (EPV == 4) mb = max(mb, w[i] & 0x7FFFFFFFu);
+        else mb = __vmaxu2(mb, w[i] & 0x7FFF7FFFu);
       }
     }
-    if (lane == 0) s[b] = bq.s;
+    if constexpr (EPV != 4) mb = max(mb & 0xFFFFu, mb >> 16);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1)
+      if (o != HALF) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+    const BlockQuant bq = block_quant(abs_max_of_bits<T>(mb));
+    int8_t* dst = q + off;
+#pragma unroll
+    for (int t = 0; t < VPR; t += VPG) {
+      float v[8];
+#pragma unroll
+      for (int g = 0; g < VPG; ++g) Vec<T>::unpack(raw[t + g], *reinterpret_cast<float(*)[EPV]>(v + g * EPV));
+      uint32_t w[2];
+      quant_pack<8>(v, bq, w);
+      if (active) {
+        if constexpr (EPV == 4) {
+          *reinterpret_cast<uint32_t*>(dst + int64_t(t) * RSTEP * C) = w[0];
+          *reinterpret_cast<uint32_t*>(dst + int64_t(t + 1) * RSTEP * C) = w[1];
+        } else {
+          *reinterpret_cast<uint2*>(dst + int64_t(t) * RSTEP * C) = make_uint2(w[0], w[1]);
+        }
+      }
+    }
+    if (active && r0 == 0 && vc % HALF == 0) s[bi * nbc + bj] = bq.s;
   }
 }
 
@@ -374,7 +399,7 @@ static int grid_for_blocks(int64_t nblocks, int sm_count) {
 
 cudaError_t launch_quantize(const void* x, int dtype, int64_t R, int64_t C, int8_t* q, float* s, int sm_count,
                             cudaStream_t st) {
-  const int grid = grid_for_blocks((R / 32) * (C / 32), sm_count);
+  const int grid = grid_for_blocks((R / 32) * ((C / 32 + 1) / 2), sm_count);  // one warp per block pair
   if (dtype == 0)
     quantize_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), R, C, q, s);
   else if (dtype == 1)
