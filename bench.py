@@ -53,7 +53,8 @@ def parse_args():
                    help="time the memory-bound kernels on the M x 4096 sweep instead of the step")
     p.add_argument("--sweep-m", type=int, nargs="*", default=[1024, 8192, 65536])
     p.add_argument("--sweep-ops", nargs="*", default=["quantize_bf16", "dequantize_bf16", "gelu_i8", "layernorm_i8",
-                                                      "gelu_i8_bwd", "layernorm_i8_bwd", "fused_fc1"])
+                                                      "gelu_i8_bwd", "layernorm_i8_bwd", "fused_fc1",
+                                                      "granularity_mse"])
     return p.parse_args()
 
 
@@ -588,9 +589,30 @@ def run_sweep(args):
         del xb, Q, D, Y, yb, ws
     if "fused_fc1" in args.sweep_ops:
         out.update(_sweep_fused_fc1(jf, flush))
+    if "granularity_mse" in args.sweep_ops:
+        out["granularity_mse"] = _granularity_mse(jf)
     assert jf.jf_device_status() == 0
     print(json.dumps({"sweep": out, "hbm_peak_gbs": peaks["hbm_gbs"], "peak_source": peak_src,
                       "l2": "flushed before every timed launch"}), flush=True)
+
+
+def _granularity_mse(jf):
+    """Quantization MSE at each scale granularity, computed on the GPU (quantize, then the fp64 error
+    sums), on the GPT2-medium fc1 activations (10 of 1024 channels x30) and on the sweep input
+    (8192 x 4096, 1% of the channels x100): the ablation of the summary's measured effects."""
+    import torch
+    from inputs import synthetic as S
+    res = {}
+    wl = __import__("inputs.synthetic", fromlist=["WORKLOADS"]).WORKLOADS[WORKLOAD]
+    host = host_inputs(wl["M"], wl["K"], wl["N"], 0, seed_weight=0)
+    cases = {"gpt2m_fc1_X": torch.from_numpy(host["x"].view(np.int16)).cuda().view(torch.bfloat16),
+             "sweep_8192x4096": torch.from_numpy(S.to_bf16_bits(S.memory_sweep_input(0, 8192, 4096)).view(np.int16))
+             .cuda().view(torch.bfloat16)}
+    for name, x in cases.items():
+        mse = {g: jf.quantization_mse(x, g) for g in ["block", "token", "channel", "tensor"]}
+        res[name] = {"mse": {g: float(f"{v:.6g}") for g, v in mse.items()},
+                     "token_over_block": round(mse["token"] / mse["block"], 2)}
+    return res
 
 
 def _sweep_fused_fc1(jf, flush):

@@ -77,8 +77,14 @@ typedef enum {
   JF_ERR_CUDA = -6,    /* a CUDA runtime or driver call failed (launch, tensor-map encode) */
   JF_ERR_TIMEOUT = -7, /* reported by jf_device_status: a kernel's bounded wait ran out */
   JF_ERR_DEVICE = -8,  /* no usable sm_100 device is current */
-  JF_ERR_WORKSPACE = -9 /* the caller's workspace is NULL, misaligned or smaller than required */
+  JF_ERR_WORKSPACE = -9, /* the caller's workspace is NULL, misaligned or smaller than required */
+  JF_ERR_ARG = -10       /* an enumerated argument (jf_granularity) is unknown */
 } jf_status;
+
+/* Scale granularity of the quantizer variants (f3): one fp32 scale per 32x32 block ([rows/32,
+ * cols/32], the Jetfire rule), per row / token ([rows]), per column / channel ([cols]), or one for
+ * the whole tensor ([1]). */
+typedef enum { JF_GRAN_BLOCK = 0, JF_GRAN_TOKEN = 1, JF_GRAN_CHANNEL = 2, JF_GRAN_TENSOR = 3 } jf_granularity;
 
 /*
  * a1. Per-block quantization (summary, "Approach": per-block scale factors, B = 32).
@@ -199,6 +205,35 @@ JF_API int64_t jf_layernorm_i8_bwd_workspace_bytes(int64_t rows, int64_t cols);
  */
 JF_API int jf_layernorm_i8_bwd_noalloc(jf_cqtensor X, jf_cqtensor dY, const float* gamma, float eps,
                                        jf_qtensor dX, float* dgamma, float* dbeta, void* stream);
+
+/*
+ * f3. Quantization at another granularity: the baselines of the summary's ablation ("Measured
+ *     effects table": per-block scales quantize activations with channel outliers more accurately
+ *     than per-token ones). The rule is that of jf_quantize_block (s = absmax / 127, IEEE quotient,
+ *     round half to even, clamp to +-127, s = 0 and codes 0 for an all-zero group), with one scale
+ *     per group of the granularity `g`. x as in jf_quantize_block; q int8 [rows, cols] (16-byte
+ *     aligned); s fp32 with jf_granular_scale_count(rows, cols, g) entries (4-byte aligned).
+ *     Codes and scales are bit-exact. JF_GRAN_BLOCK is jf_quantize_block.
+ */
+JF_API int jf_quantize_granular(const void* x, jf_dtype dt, int64_t rows, int64_t cols, jf_granularity g, int8_t* q,
+                                float* s, void* stream);
+
+/* Number of scales of a [rows, cols] tensor at granularity g, or -1 for an invalid shape or g. */
+JF_API int64_t jf_granular_scale_count(int64_t rows, int64_t cols, jf_granularity g);
+
+/* f3. y = fp32(q) * s of the element's group, rounded to nearest even into dt (bit-exact). */
+JF_API int jf_dequantize_granular(const int8_t* q, const float* s, int64_t rows, int64_t cols, jf_granularity g,
+                                  void* y, jf_dtype dt, void* stream);
+
+/*
+ * f3. The error of a quantization (the summary's accuracy metric behind the ablation): writes
+ *     sums[0] = sum over elements of (x - q s)^2 and sums[1] = sum of x^2, in fp64, to the device
+ *     array `sums` (2 doubles, 8-byte aligned); x, q and s as above, all exact in fp64, so only the
+ *     order of the fp64 additions (unspecified) affects the result. The mean squared error is
+ *     sums[0] / (rows * cols).
+ */
+JF_API int jf_quantization_error(const void* x, jf_dtype dt, const int8_t* q, const float* s, int64_t rows,
+                                 int64_t cols, jf_granularity g, double* sums, void* stream);
 
 /* Static description of a status code (never NULL). */
 JF_API const char* jf_strerror(int status);

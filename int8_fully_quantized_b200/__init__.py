@@ -22,25 +22,29 @@ from . import build_lib
 from .build_lib import LIB_PATH
 
 __all__ = [
-    "QTensor", "JetfireError", "load_library", "empty_qtensor", "jf_quantize_block", "jf_dequantize_block",
-    "jf_linear_fwd", "jf_linear_fwd_gelu", "jf_linear_dgrad", "jf_linear_wgrad", "jf_gelu_i8", "jf_layernorm_i8",
-    "jf_gelu_i8_bwd", "jf_layernorm_i8_bwd", "jf_layernorm_i8_bwd_workspace_bytes", "jf_layernorm_i8_bwd_noalloc",
-    "gelu_i8_bwd",
-    "layernorm_i8_bwd", "jf_strerror", "jf_device_status", "jf_sm_count", "quantize_block", "dequantize_block",
-    "linear_fwd",
-    "linear_fwd_gelu", "linear_dgrad",
-    "linear_wgrad", "gelu_i8", "layernorm_i8", "EXPORTED_SYMBOLS", "JF_F32", "JF_BF16", "JF_F16",
+    "QTensor", "JetfireError", "load_library", "empty_qtensor", "EXPORTED_SYMBOLS", "JF_F32", "JF_BF16", "JF_F16",
+    "GRANULARITY",
+    # C ABI, one wrapper per entry point
+    "jf_quantize_block", "jf_dequantize_block", "jf_linear_fwd", "jf_linear_fwd_gelu", "jf_linear_dgrad",
+    "jf_linear_wgrad", "jf_gelu_i8", "jf_layernorm_i8", "jf_gelu_i8_bwd", "jf_layernorm_i8_bwd",
+    "jf_layernorm_i8_bwd_workspace_bytes", "jf_layernorm_i8_bwd_noalloc", "jf_quantize_granular",
+    "jf_dequantize_granular", "jf_quantization_error", "jf_granular_scale_count", "jf_strerror",
+    "jf_device_status", "jf_sm_count",
+    # allocating helpers
+    "quantize_block", "dequantize_block", "linear_fwd", "linear_fwd_gelu", "linear_dgrad", "linear_wgrad",
+    "gelu_i8", "layernorm_i8", "gelu_i8_bwd", "layernorm_i8_bwd", "quantize_granular", "quantization_mse",
 ]
 
 JF_F32, JF_BF16, JF_F16 = 0, 1, 2
+GRANULARITY = {"block": 0, "token": 1, "channel": 2, "tensor": 3}
 _DTYPES = {torch.float32: JF_F32, torch.bfloat16: JF_BF16, torch.float16: JF_F16}
 
 EXPORTED_SYMBOLS = (
     "jf_quantize_block", "jf_dequantize_block", "jf_linear_fwd", "jf_linear_fwd_gelu", "jf_linear_dgrad",
     "jf_linear_wgrad",
     "jf_gelu_i8", "jf_layernorm_i8", "jf_gelu_i8_bwd", "jf_layernorm_i8_bwd", "jf_layernorm_i8_bwd_workspace_bytes",
-    "jf_layernorm_i8_bwd_noalloc",
-    "jf_strerror", "jf_device_status", "jf_sm_count",
+    "jf_layernorm_i8_bwd_noalloc", "jf_quantize_granular", "jf_dequantize_granular", "jf_quantization_error",
+    "jf_granular_scale_count", "jf_strerror", "jf_device_status", "jf_sm_count",
 )
 
 
@@ -85,6 +89,10 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.jf_layernorm_i8_bwd.argtypes = [_CQ, _CQ, vp, ctypes.c_float, _Q, vp, vp, vp, i64, vp]
     lib.jf_layernorm_i8_bwd_workspace_bytes.argtypes = [i64, i64]
     lib.jf_layernorm_i8_bwd_noalloc.argtypes = [_CQ, _CQ, vp, ctypes.c_float, _Q, vp, vp, vp]
+    lib.jf_quantize_granular.argtypes = [vp, i32, i64, i64, i32, vp, vp, vp]
+    lib.jf_dequantize_granular.argtypes = [vp, vp, i64, i64, i32, vp, i32, vp]
+    lib.jf_quantization_error.argtypes = [vp, i32, vp, vp, i64, i64, i32, vp, vp]
+    lib.jf_granular_scale_count.argtypes = [i64, i64, i32]
     lib.jf_strerror.argtypes = [i32]
     lib.jf_strerror.restype = ctypes.c_char_p
     lib.jf_device_status.argtypes = [vp]
@@ -93,6 +101,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         if name != "jf_strerror":
             getattr(lib, name).restype = ctypes.c_int
     lib.jf_layernorm_i8_bwd_workspace_bytes.restype = i64
+    lib.jf_granular_scale_count.restype = i64
     _lib = lib
     return lib
 
@@ -224,6 +233,46 @@ def jf_layernorm_i8_bwd_noalloc(X: QTensor, dY: QTensor, gamma: torch.Tensor, ep
     lib = load_library()
     _check(lib.jf_layernorm_i8_bwd_noalloc(_cq(X), _cq(dY), _ptr(gamma), ctypes.c_float(eps), _q(dX, X.rows, X.cols),
                                            _ptr(dgamma), _ptr(dbeta), _stream(stream)), "jf_layernorm_i8_bwd_noalloc")
+
+
+def jf_granular_scale_count(rows: int, cols: int, g: int) -> int:
+    return int(load_library().jf_granular_scale_count(rows, cols, g))
+
+
+def jf_quantize_granular(x: torch.Tensor, g: int, q: torch.Tensor, s: torch.Tensor, stream=None) -> None:
+    lib = load_library()
+    _check(lib.jf_quantize_granular(_ptr(x), _DTYPES[x.dtype], x.shape[0], x.shape[1], g, _ptr(q), _ptr(s),
+                                    _stream(stream)), "jf_quantize_granular")
+
+
+def jf_dequantize_granular(q: torch.Tensor, s: torch.Tensor, g: int, y: torch.Tensor, stream=None) -> None:
+    lib = load_library()
+    _check(lib.jf_dequantize_granular(_ptr(q), _ptr(s), q.shape[0], q.shape[1], g, _ptr(y), _DTYPES[y.dtype],
+                                      _stream(stream)), "jf_dequantize_granular")
+
+
+def jf_quantization_error(x: torch.Tensor, q: torch.Tensor, s: torch.Tensor, g: int, sums: torch.Tensor,
+                          stream=None) -> None:
+    lib = load_library()
+    _check(lib.jf_quantization_error(_ptr(x), _DTYPES[x.dtype], _ptr(q), _ptr(s), x.shape[0], x.shape[1], g,
+                                     _ptr(sums), _stream(stream)), "jf_quantization_error")
+
+
+def quantize_granular(x: torch.Tensor, granularity: str, stream=None):
+    """(codes, scales) of x at one granularity: "block", "token", "channel" or "tensor"."""
+    g = GRANULARITY[granularity]
+    q = torch.empty(x.shape, dtype=torch.int8, device=x.device)
+    s = torch.empty(jf_granular_scale_count(x.shape[0], x.shape[1], g), dtype=torch.float32, device=x.device)
+    jf_quantize_granular(x, g, q, s, stream)
+    return q, s
+
+
+def quantization_mse(x: torch.Tensor, granularity: str, stream=None) -> float:
+    """Mean squared error of quantize -> dequantize at one granularity, computed on the GPU."""
+    q, s = quantize_granular(x, granularity, stream)
+    sums = torch.empty(2, dtype=torch.float64, device=x.device)
+    jf_quantization_error(x, q, s, GRANULARITY[granularity], sums, stream)
+    return float(sums[0].item()) / x.numel()
 
 
 def jf_strerror(status: int) -> str:

@@ -318,6 +318,74 @@ int jf_layernorm_i8_bwd_noalloc(jf_cqtensor X, jf_cqtensor dY, const float* gamm
   return jf_layernorm_i8_bwd(X, dY, gamma, eps, dX, dgamma, dbeta, scratch, jf::kLnBwdScratchBytes, stream);
 }
 
+int64_t jf_granular_scale_count(int64_t rows, int64_t cols, jf_granularity g) {
+  if (!dims_ok(rows, cols)) return -1;
+  switch (g) {
+    case JF_GRAN_BLOCK: return (rows / 32) * (cols / 32);
+    case JF_GRAN_TOKEN: return rows;
+    case JF_GRAN_CHANNEL: return cols;
+    case JF_GRAN_TENSOR: return 1;
+    default: return -1;
+  }
+}
+
+namespace {
+bool gran_ok(jf_granularity g) { return g == JF_GRAN_BLOCK || g == JF_GRAN_TOKEN || g == JF_GRAN_CHANNEL || g == JF_GRAN_TENSOR; }
+}  // namespace
+
+int jf_quantize_granular(const void* x, jf_dtype dt, int64_t rows, int64_t cols, jf_granularity g, int8_t* q,
+                         float* s, void* stream) {
+  if (dt != JF_F32 && dt != JF_BF16 && dt != JF_F16) return JF_ERR_DTYPE;
+  if (!gran_ok(g)) return JF_ERR_ARG;
+  if (!dims_ok(rows, cols)) return JF_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return JF_OK;
+  if (x == nullptr || q == nullptr || s == nullptr) return JF_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(s, 4)) return JF_ERR_ALIGN;
+  const int64_t nx = rows * cols * elem_size(dt), ns = jf_granular_scale_count(rows, cols, g) * 4;
+  if (overlap(q, rows * cols, x, nx) || overlap(s, ns, x, nx) || overlap(q, rows * cols, s, ns)) return JF_ERR_ALIAS;
+  const DevInfo d = device_info();
+  if (!d.ok) return JF_ERR_DEVICE;
+  return cuda_status(jf::launch_quantize_granular(x, int(dt), rows, cols, int(g), q, s, d.sm_count,
+                                                  static_cast<cudaStream_t>(stream)));
+}
+
+int jf_dequantize_granular(const int8_t* q, const float* s, int64_t rows, int64_t cols, jf_granularity g, void* y,
+                           jf_dtype dt, void* stream) {
+  if (dt != JF_F32 && dt != JF_BF16 && dt != JF_F16) return JF_ERR_DTYPE;
+  if (!gran_ok(g)) return JF_ERR_ARG;
+  if (!dims_ok(rows, cols)) return JF_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return JF_OK;
+  if (q == nullptr || s == nullptr || y == nullptr) return JF_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(s, 4) || !aligned(y, 16)) return JF_ERR_ALIGN;
+  const int64_t ny = rows * cols * elem_size(dt), ns = jf_granular_scale_count(rows, cols, g) * 4;
+  if (overlap(y, ny, q, rows * cols) || overlap(y, ny, s, ns)) return JF_ERR_ALIAS;
+  const DevInfo d = device_info();
+  if (!d.ok) return JF_ERR_DEVICE;
+  return cuda_status(jf::launch_dequantize_granular(q, s, rows, cols, int(g), y, int(dt), d.sm_count,
+                                                    static_cast<cudaStream_t>(stream)));
+}
+
+int jf_quantization_error(const void* x, jf_dtype dt, const int8_t* q, const float* s, int64_t rows, int64_t cols,
+                          jf_granularity g, double* sums, void* stream) {
+  if (dt != JF_F32 && dt != JF_BF16 && dt != JF_F16) return JF_ERR_DTYPE;
+  if (!gran_ok(g)) return JF_ERR_ARG;
+  if (!dims_ok(rows, cols)) return JF_ERR_SHAPE;
+  if (sums == nullptr) return JF_ERR_NULL;
+  if (!aligned(sums, 8)) return JF_ERR_ALIGN;
+  const int64_t nx = rows * cols * elem_size(dt), ns = jf_granular_scale_count(rows, cols, g) * 4;
+  if (rows != 0 && cols != 0) {
+    if (x == nullptr || q == nullptr || s == nullptr) return JF_ERR_NULL;
+    if (!aligned(x, 16) || !aligned(q, 16) || !aligned(s, 4)) return JF_ERR_ALIGN;
+    if (overlap(sums, 16, x, nx) || overlap(sums, 16, q, rows * cols) || overlap(sums, 16, s, ns)) return JF_ERR_ALIAS;
+  }
+  const DevInfo d = device_info();
+  if (!d.ok) return JF_ERR_DEVICE;
+  if (rows == 0 || cols == 0)
+    return cuda_status(cudaMemsetAsync(sums, 0, 2 * sizeof(double), static_cast<cudaStream_t>(stream)));
+  return cuda_status(jf::launch_quant_error(x, int(dt), q, s, rows, cols, int(g), sums, d.sm_count,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
 const char* jf_strerror(int status) {
   switch (status) {
     case JF_OK: return "ok";
@@ -330,6 +398,7 @@ const char* jf_strerror(int status) {
     case JF_ERR_TIMEOUT: return "a kernel's bounded wait timed out; outputs are undefined";
     case JF_ERR_DEVICE: return "no usable sm_100 (B200) device is current";
     case JF_ERR_WORKSPACE: return "workspace is NULL, not 16-byte aligned or smaller than the size asked for";
+    case JF_ERR_ARG: return "unknown granularity (or other enumerated argument)";
     default: return "unknown status";
   }
 }

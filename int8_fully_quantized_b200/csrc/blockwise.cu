@@ -16,68 +16,9 @@
 #include "kernels.h"
 #include "ptx.cuh"
 #include "quant.cuh"
+#include "vec.cuh"
 
 namespace jf {
-
-// ---------------------------------------------------------------------------------------------
-// element unpack / pack helpers for the 16-byte vectors the kernels move
-// ---------------------------------------------------------------------------------------------
-template <typename T>
-struct Vec;
-template <>
-struct Vec<float> {
-  static constexpr int kElems = 4;
-  __device__ static void unpack(const uint4& v, float (&f)[4]) {
-    f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
-    f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
-  }
-  __device__ static uint4 pack(const float (&f)[4]) {
-    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]), __float_as_uint(f[3]));
-  }
-};
-template <>
-struct Vec<__nv_bfloat16> {
-  static constexpr int kElems = 8;
-  __device__ static void unpack(const uint4& v, float (&f)[8]) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {  // bf16 is the upper half of an fp32: exact widening
-      f[2 * i] = __uint_as_float(w[i] << 16);
-      f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-  }
-  __device__ static uint4 pack(const float (&f)[8]) {
-    uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
-      w[i] = *reinterpret_cast<uint32_t*>(&h);
-    }
-    return make_uint4(w[0], w[1], w[2], w[3]);
-  }
-};
-template <>
-struct Vec<__half> {
-  static constexpr int kElems = 8;
-  __device__ static void unpack(const uint4& v, float (&f)[8]) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float2 p = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
-      f[2 * i] = p.x;
-      f[2 * i + 1] = p.y;
-    }
-  }
-  __device__ static uint4 pack(const float (&f)[8]) {
-    uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      __half2 h = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
-      w[i] = *reinterpret_cast<uint32_t*>(&h);
-    }
-    return make_uint4(w[0], w[1], w[2], w[3]);
-  }
-};
 
 // ---------------------------------------------------------------------------------------------
 // a1: quantize. One warp per pair of horizontally adjacent 32x32 blocks (a 32 x 64 tile), so that
@@ -90,17 +31,6 @@ struct Vec<__half> {
 // cleared), reduced over the 16 lanes of the lane's block, and the values are unpacked and quantized
 // eight at a time. When the number of block columns is odd the last pair holds one block.
 // ---------------------------------------------------------------------------------------------
-template <typename T>
-__device__ __forceinline__ float abs_max_of_bits(uint32_t m);  // m: the largest |x| bit pattern
-template <>
-__device__ __forceinline__ float abs_max_of_bits<float>(uint32_t m) { return __uint_as_float(m); }
-template <>
-__device__ __forceinline__ float abs_max_of_bits<__nv_bfloat16>(uint32_t m) { return __uint_as_float(m << 16); }
-template <>
-__device__ __forceinline__ float abs_max_of_bits<__half>(uint32_t m) {
-  return __half2float(__ushort_as_half(static_cast<unsigned short>(m)));
-}
-
 template <typename T>
 __global__ void __launch_bounds__(256, 3) quantize_kernel(const T* __restrict__ x, int64_t R, int64_t C,
                                                           int8_t* __restrict__ q, float* __restrict__ s) {

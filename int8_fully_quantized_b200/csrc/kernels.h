@@ -12,6 +12,16 @@ cudaError_t launch_dequantize(const int8_t* q, const float* s, int64_t R, int64_
                               int sm_count, cudaStream_t st);
 cudaError_t launch_gelu_i8(const int8_t* q, const float* s, int64_t R, int64_t C, int8_t* qo, float* so,
                            int sm_count, cudaStream_t st);
+// Granularity variants of the quantizer and the quantization-error sums (granular.cu). Scales:
+// block [R/32, C/32], token [R], channel [C], tensor [1].
+enum Granularity { kGranBlock = 0, kGranToken = 1, kGranChannel = 2, kGranTensor = 3 };
+cudaError_t launch_quantize_granular(const void* x, int dtype, int64_t R, int64_t C, int g, int8_t* q, float* s,
+                                     int sm_count, cudaStream_t st);
+cudaError_t launch_dequantize_granular(const int8_t* q, const float* s, int64_t R, int64_t C, int g, void* y,
+                                       int dtype, int sm_count, cudaStream_t st);
+cudaError_t launch_quant_error(const void* x, int dtype, const int8_t* q, const float* s, int64_t R, int64_t C, int g,
+                               double* sums, int sm_count, cudaStream_t st);
+
 // INT8 backward of GELU_i8 and LayerNorm_i8 (backward.cu). `part` is the fp32 workspace of
 // per-CTA column sums, [ln_bwd_ctas(R)][2][H]; null when neither dgamma nor dbeta is wanted.
 constexpr int64_t kLnBwdMaxCtas = 444;   // three resident CTAs on each of 148 SMs

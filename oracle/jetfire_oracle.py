@@ -42,7 +42,7 @@ QMAX = 127
 
 __all__ = [
     "BLOCK", "QMAX", "bf16_bits_to_f32", "f32_to_bf16_bits", "quantize", "quantize_block",
-    "dequantize_block", "block_scale_grid", "linear_fwd", "linear_fwd_gelu", "linear_dgrad", "linear_wgrad",
+    "dequantize_block", "dequantize", "block_scale_grid", "linear_fwd", "linear_fwd_gelu", "linear_dgrad", "linear_wgrad",
     "requantize", "gelu_i8", "layernorm_i8", "gelu_f64", "quantization_mse", "gelu_grad_f64",
     "gelu_i8_bwd", "layernorm_i8_bwd",
 ]
@@ -107,7 +107,13 @@ def dequantize_block(q: np.ndarray, s: np.ndarray, out: str = "f32") -> np.ndarr
     """y = fp32(q) * s (one fp32 rounding), then round-to-nearest-even to the output dtype.
 
     ``out``: "f32" (fp32 array), "bf16" (uint16 bit pattern) or "f16" (float16 array)."""
-    y = (np.asarray(q).astype(np.float32) * block_scale_grid(s)).astype(np.float32)
+    return dequantize(q, s, BLOCK, BLOCK, out)
+
+
+def dequantize(q: np.ndarray, s: np.ndarray, block_rows: int, block_cols: int, out: str = "f32") -> np.ndarray:
+    """dequantize_block for any block shape (the granularity variants: (1, C) per token, (R, 1) per
+    channel, (R, C) per tensor), with s [R/block_rows, C/block_cols]."""
+    y = (np.asarray(q).astype(np.float32) * block_scale_grid(s, block_rows, block_cols)).astype(np.float32)
     if out == "f32":
         return y
     if out == "bf16":

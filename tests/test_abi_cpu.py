@@ -109,6 +109,12 @@ def test_host_validation_rejects_bad_arguments(lib):
     # the allocation-free backward refuses shapes whose column sums exceed its 16 MiB static scratch
     big = jf._CQ(1 << 20, 1 << 22, 32768, 8192)
     assert lib.jf_layernorm_i8_bwd_noalloc(big, big, g, f, jf._Q(1 << 28, 1 << 30, 32768, 8192), dg, db, None) == -9
+    # granularity variants: unknown granularity, scale counts
+    assert lib.jf_quantize_granular(fake, 1, 32, 64, 7, fake, fake, None) == -10
+    assert [lib.jf_granular_scale_count(64, 96, g) for g in range(4)] == [6, 64, 96, 1]
+    assert lib.jf_granular_scale_count(64, 96, 9) == -1
+    assert lib.jf_quantization_error(fake, 1, fake, fake, 32, 32, 1, None, None) == -1
+    assert lib.jf_dequantize_granular(fake, fake, 32, 32, 2, vp(1 << 20), 1, None) == -5
     # LayerNorm needs gamma/beta
     assert lib.jf_layernorm_i8(jf._CQ(1 << 20, 1 << 22, 32, 64), None, fake, ctypes.c_float(1e-5),
                                jf._Q(1 << 28, 1 << 30, 32, 64), None) == -1

@@ -502,3 +502,33 @@ def test_layernorm_i8_bwd_vs_torch_autograd_and_invariants():
     xh = (xd - xd.mean(1, keepdims=True)) / np.sqrt(xd.var(1, keepdims=True))
     dx0 = dx0.astype(np.float64)
     assert np.all(np.abs((dx0 * xh).sum(1)) <= 1e-6 * np.abs(dx0 * xh).sum(1))
+
+
+# ---------------------------------------------------------------------------------------------
+# f3: granularity variants
+# ---------------------------------------------------------------------------------------------
+def test_granularity_variants_relations_and_bounds():
+    """Per-channel quantization is per-token quantization of the transpose (bit for bit); per-token
+    quantization of each row alone is per-tensor quantization of that row; every group reaches
+    |q| = 127 and every element meets the rounding bound |x - q s| <= s/2 (1 + 2^-22)."""
+    rng = np.random.default_rng(40)
+    x = S.activation(rng, 96, 160, 3, 40.0)
+    x[5] = 0.0                                     # an all-zero row: s = 0, codes 0
+    R, C = x.shape
+    qt, st = O.quantize(x, 1, C)
+    qc, sc = O.quantize(x.T.copy(), 1, R)
+    qch, sch = O.quantize(x, R, 1)
+    assert np.array_equal(qch, qc.T) and np.array_equal(sch.ravel(), sc.ravel())
+    for r in (0, 5, 17, 95):
+        q1, s1 = O.quantize(x[r:r + 1], 1, C)
+        assert np.array_equal(q1[0], qt[r]) and s1[0, 0] == st[r, 0]
+    assert st[5, 0] == 0 and not qt[5].any()
+    for (br, bc), (q, s) in {(1, C): (qt, st), (R, 1): (qch, sch), (R, C): O.quantize(x, R, C)}.items():
+        sg = O.block_scale_grid(s, br, bc).astype(np.float64)
+        err = np.abs(x.astype(np.float64) - q.astype(np.float64) * sg)
+        assert np.all(err <= sg / 2 * (1 + 2.0 ** -22))
+        qa = np.abs(q.astype(np.int32)).reshape(R // br, br, C // bc, bc).max(axis=(1, 3))
+        assert np.all((qa == 127) | (s == 0))
+    # dequantize at any granularity is fp32(q) * s of the element's group
+    y = O.dequantize(qt, st, 1, C)
+    assert np.array_equal(y, (qt.astype(np.float32) * st.astype(np.float32)).astype(np.float32))
