@@ -139,59 +139,112 @@ __global__ void __launch_bounds__(256, 4) dequantize_kernel(const int8_t* __rest
 }
 
 // ---------------------------------------------------------------------------------------------
-// a6: GELU_i8. One warp per block; the block is 64 16-byte chunks, lane l takes chunks l and
-// l + 32, i.e. columns 16 (l % 2) .. +15 of rows l / 2 and 16 + l / 2.
-// GELU is evaluated by gelu_f32 (act.cuh), in its erfc form.
+// a6: GELU_i8. One warp per pair of horizontally adjacent blocks (a 32 x 64 tile), so that every
+// store writes whole 64-byte row segments (see quantize). Lane l takes the 16-byte vector l % 4 of
+// rows l / 4 + 8 t (t = 0..3): 64 codes, all of block (l % 4) / 2 of the pair.
+// A block's input has at most 255 distinct values q * s, so its output is a function of the input
+// code alone:
+//   1. value table: GELU of every code of both blocks. One erfc serves a code and its negation:
+//      with e = erfc(x / sqrt 2) for x = |q| s (erfc_nonneg, act.cuh), GELU(x) = 0.5 x (2 - e) and
+//      GELU(-x) = -0.5 x e (the erfc form of GELU, which keeps its relative accuracy for negative x);
+//   2. block absmax without touching the elements: GELU is increasing for x > -0.75 and
+//      |GELU(x)| < 0.17 for x < 0, so when GELU(qmax s) >= 0.17 (qmax: the largest code, a bytewise
+//      integer max) it is the absmax; otherwise (rare) the lanes take the max over their lookups;
+//   3. code table: the quantized code of every table value (256 per block, the same rule as
+//      everywhere), so that each element costs one byte lookup.
 // ---------------------------------------------------------------------------------------------
-
 constexpr int kGeluWarps = 8;
+constexpr float kGeluNegBound = 0.17f;  // > max |GELU(x)| over x < 0 (0.16997 at x = -0.7518)
 
-__global__ void __launch_bounds__(32 * kGeluWarps, 4) gelu_i8_kernel(const int8_t* __restrict__ q,
+__global__ void __launch_bounds__(32 * kGeluWarps, 3) gelu_i8_kernel(const int8_t* __restrict__ q,
                                                                     const float* __restrict__ s, int64_t R,
                                                                     int64_t C, int8_t* __restrict__ qo,
                                                                     float* __restrict__ so) {
-  // A block's input has at most 255 distinct values q * s, so each warp first tabulates GELU of all
-  // of them (8 evaluations per lane instead of 32) and then looks its 32 values up; the results are
-  // the same as evaluating GELU per element.
-  __shared__ float table[kGeluWarps][256];
+  __shared__ float table[kGeluWarps][2][256];
+  __shared__ __align__(16) uint8_t codes[kGeluWarps][2][256];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  float* tab = table[wib];
   const int64_t nbc = C >> 5;
-  const int64_t nblocks = (R >> 5) * nbc;
+  const int64_t npc = (nbc + 1) >> 1;   // block pairs per block row
+  const int64_t npairs = (R >> 5) * npc;
   const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
-  const int r0 = lane >> 1, c0 = (lane & 1) * 16;
-  for (int64_t b = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; b < nblocks; b += nwarps) {
-    const int64_t bi = b / nbc, bj = b - bi * nbc;
-    const float sc = __ldg(s + b);
-    const int64_t off = (bi * 32 + r0) * C + bj * 32 + c0;
-    const uint4 a0 = ld_stream_v4(q + off);
-    const uint4 a1 = ld_stream_v4(q + off + 16 * C);
-    // table[u] = GELU(fp32(u - 128) * s) for u = 1..255 (code u - 128)
+  const int vc = lane & 3, r0 = lane >> 2, half = vc >> 1;
+  const float* tab = table[wib][half];
+  const uint8_t* ctab = codes[wib][half];
+  // table-building role: lanes 0-15 build block 0, lanes 16-31 block 1
+  const int tb = lane >> 4, k = lane & 15;
+  for (int64_t p = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; p < npairs; p += nwarps) {
+    const int64_t bi = p / npc, pj = p - bi * npc;
+    const int64_t b0 = bi * nbc + 2 * pj;             // first block of the pair
+    const bool has1 = 2 * pj + 1 < nbc;               // the pair's second block exists
+    const bool active = half == 0 || has1;
+    const int64_t off = (bi * 32 + r0) * C + pj * 64 + vc * 16;
+    uint4 a[4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int u = lane + 32 * j;
-      tab[u] = gelu_f32(float(u - 128) * sc);
+    for (int t = 0; t < 4; ++t) a[t] = active ? ld_stream_v4(q + off + int64_t(t) * 8 * C) : make_uint4(0u, 0u, 0u, 0u);
+    // 1. value tables (index = code + 128)
+    {
+      float* tw = table[wib][tb];
+      const float sc = (tb == 0 || has1) ? __ldg(s + b0 + tb) : 0.0f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int m = k + 16 * j;                      // |code| 0..127
+        const float x = float(m) * sc;
+        const float e = erfc_nonneg(x * 0.70710678118654752440f);
+        tw[128 - m] = -0.5f * x * e;                   // code -m
+        tw[128 + m] = 0.5f * x * (2.0f - e);           // code +m (for m = 0 this +0 is the entry kept)
+      }
+      if (k == 0) tw[0] = -0.5f * (128.0f * sc) * erfc_nonneg(128.0f * sc * 0.70710678118654752440f);  // code -128
+    }
+    // 2. block absmax: the largest code of the lane's block (bytewise signed max), then its GELU
+    uint32_t mx = 0x80808080u;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) mx = __vmaxs4(__vmaxs4(mx, a[t].x), __vmaxs4(__vmaxs4(a[t].y, a[t].z), a[t].w));
+    int qmax = max(max(int(int8_t(mx)), int(int8_t(mx >> 8))), max(int(int8_t(mx >> 16)), int(int8_t(mx >> 24))));
+    qmax = max(qmax, __shfl_xor_sync(0xffffffffu, qmax, 1));
+    qmax = max(qmax, __shfl_xor_sync(0xffffffffu, qmax, 4));
+    qmax = max(qmax, __shfl_xor_sync(0xffffffffu, qmax, 8));
+    qmax = max(qmax, __shfl_xor_sync(0xffffffffu, qmax, 16));
+    __syncwarp();
+    float amax = tab[qmax + 128];
+    if (__any_sync(0xffffffffu, !(amax >= kGeluNegBound))) {
+      float m = 0.0f;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const uint32_t w[4] = {a[t].x ^ 0x80808080u, a[t].y ^ 0x80808080u, a[t].z ^ 0x80808080u, a[t].w ^ 0x80808080u};
+#pragma unroll
+        for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(tab[(w[i >> 2] >> (8 * (i & 3))) & 0xFFu]));
+      }
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+      amax = m;
+    }
+    // 3. code tables: lane k of each half quantizes entries k + 16 i of its block's table (consecutive
+    //    lanes touch consecutive words: no shared-memory bank conflicts)
+    {
+      const float amax_tb = __shfl_sync(0xffffffffu, amax, tb == 0 ? 0 : 2);  // lane 0: block 0, lane 2: block 1
+      const BlockQuant bt = block_quant(amax_tb);
+      float v[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = table[wib][tb][k + 16 * i];
+      uint32_t o[4];
+      quant_pack<16>(v, bt, o);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) codes[wib][tb][k + 16 * i] = uint8_t(o[i >> 2] >> (8 * (i & 3)));
+      if (r0 == 0 && (vc & 1) == 0 && active) so[b0 + half] = __fdiv_rn(amax, kQMax);
     }
     __syncwarp();
-    const uint32_t w[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-    float v[32];
-    float m = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t u = w[i] ^ 0x80808080u;  // code + 128 in each byte
+    for (int t = 0; t < 4; ++t) {
+      const uint32_t w[4] = {a[t].x ^ 0x80808080u, a[t].y ^ 0x80808080u, a[t].z ^ 0x80808080u, a[t].w ^ 0x80808080u};
+      uint32_t o[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        v[4 * i + j] = tab[(u >> (8 * j)) & 0xFFu];
-        m = fmaxf(m, fabsf(v[4 * i + j]));
-      }
+      for (int i = 0; i < 4; ++i)
+        o[i] = pack4(ctab[w[i] & 0xFFu], ctab[(w[i] >> 8) & 0xFFu], ctab[(w[i] >> 16) & 0xFFu], ctab[w[i] >> 24]);
+      if (active) *reinterpret_cast<uint4*>(qo + off + int64_t(t) * 8 * C) = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    __syncwarp();  // the table is rewritten for the next block only after every lane has read it
-    const BlockQuant bq = block_quant(warp_max_nonneg(m));
-    uint32_t o[8];
-    quant_pack<32>(v, bq, o);
-    *reinterpret_cast<uint4*>(qo + off) = make_uint4(o[0], o[1], o[2], o[3]);
-    *reinterpret_cast<uint4*>(qo + off + 16 * C) = make_uint4(o[4], o[5], o[6], o[7]);
-    if (lane == 0) so[b] = bq.s;
+    __syncwarp();  // the tables are rewritten for the next pair only after every lane has read them
   }
 }
 
@@ -353,7 +406,7 @@ cudaError_t launch_dequantize(const int8_t* q, const float* s, int64_t R, int64_
 
 cudaError_t launch_gelu_i8(const int8_t* q, const float* s, int64_t R, int64_t C, int8_t* qo, float* so,
                            int sm_count, cudaStream_t st) {
-  const int grid = grid_for_blocks((R / 32) * (C / 32), sm_count);
+  const int grid = grid_for_blocks((R / 32) * ((C / 32 + 1) / 2), sm_count);  // one warp per block pair
   gelu_i8_kernel<<<grid, 32 * kGeluWarps, 0, st>>>(q, s, R, C, qo, so);
   return cudaGetLastError();
 }
