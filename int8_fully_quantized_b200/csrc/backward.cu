@@ -103,6 +103,7 @@ __global__ void __launch_bounds__(kLnbThreads, 3) layernorm_i8_bwd_kernel(
   extern __shared__ float s_acc[];  // [2][H] column sums of dy xhat and dy over this CTA's strips
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t nbc = H >> 5;
+  const uint64_t keep = l2_policy_evict_last(), stream = l2_policy_evict_first();
   if (part != nullptr)
     for (int64_t c = threadIdx.x; c < 2 * H; c += kLnbThreads) s_acc[c] = 0.0f;
   for (int64_t strip = blockIdx.x; strip < (R >> 5); strip += gridDim.x) {
@@ -123,8 +124,8 @@ __global__ void __launch_bounds__(kLnbThreads, 3) layernorm_i8_bwd_kernel(
         for (int u = 0; u < kUnroll; ++u) {
           const int64_t ch = ch0 + 32 * u;
           if (ch < (H >> 4)) {
-            av[u] = ld_stream_v4(xrow + ch * 16);
-            dv[u] = ld_stream_v4(drow + ch * 16);
+            av[u] = ld_v4_policy(xrow + ch * 16, keep);  // read again in phase 2: keep it in L2
+            dv[u] = ld_v4_policy(drow + ch * 16, keep);
             scx[u] = __ldg(xss + (ch >> 1));
             scd[u] = __ldg(dss + (ch >> 1));
           } else {
@@ -192,8 +193,8 @@ __global__ void __launch_bounds__(kLnbThreads, 3) layernorm_i8_bwd_kernel(
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int64_t off = int64_t(rg + 4 * i) * H + col;
-        wx[i] = ld_stream_b32(xstrip + off);
-        wd[i] = ld_stream_b32(dstrip + off);
+        wx[i] = ld_b32_policy(xstrip + off, stream);
+        wd[i] = ld_b32_policy(dstrip + off, stream);
       }
       float v[32], pgam[4] = {0.0f, 0.0f, 0.0f, 0.0f}, pbet[4] = {0.0f, 0.0f, 0.0f, 0.0f};
       float m = 0.0f;
@@ -219,7 +220,7 @@ __global__ void __launch_bounds__(kLnbThreads, 3) layernorm_i8_bwd_kernel(
       quant_pack<32>(v, bq, o);
       int8_t* dst = qo + strip * 32 * H;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) *reinterpret_cast<uint32_t*>(dst + int64_t(rg + 4 * i) * H + col) = o[i];
+      for (int i = 0; i < 8; ++i) st_b32_policy(dst + int64_t(rg + 4 * i) * H + col, o[i], stream);
       if (lane == 0) so[strip * nbc + bj] = bq.s;
       if (part != nullptr) {
 #pragma unroll

@@ -272,6 +272,7 @@ __global__ void __launch_bounds__(kLnThreads, 2) layernorm_i8_kernel(const int8_
   const int64_t nbc = H >> 5;
   const int8_t* qs = q + strip * 32 * H;
   const float* ss = s + strip * nbc;
+  const uint64_t keep = l2_policy_evict_last(), stream = l2_policy_evict_first();
   for (int rw = warp; rw < 32; rw += kLnThreads / 32) {
     const int8_t* row = qs + int64_t(rw) * H;
     double sum = 0.0, sq = 0.0;
@@ -283,7 +284,7 @@ __global__ void __launch_bounds__(kLnThreads, 2) layernorm_i8_kernel(const int8_
       for (int u = 0; u < kUnroll; ++u) {
         const int64_t ch = ch0 + 32 * u;
         if (ch < (H >> 4)) {
-          av[u] = ld_stream_v4(row + ch * 16);
+          av[u] = ld_v4_policy(row + ch * 16, keep);  // read again in phase 2: keep it in L2
           scv[u] = __ldg(ss + (ch >> 1));
         } else {
           av[u] = make_uint4(0u, 0u, 0u, 0u);
@@ -331,8 +332,8 @@ __global__ void __launch_bounds__(kLnThreads, 2) layernorm_i8_kernel(const int8_
   for (int64_t bj = warp; bj < nbc; bj += kLnThreads / 32) {
     const int64_t off = int64_t(r0) * H + bj * 32 + c0;
     const float sc = __ldg(ss + bj);
-    const uint4 a0 = *reinterpret_cast<const uint4*>(qs + off);
-    const uint4 a1 = *reinterpret_cast<const uint4*>(qs + off + 16 * H);
+    const uint4 a0 = ld_v4_policy(qs + off, stream);
+    const uint4 a1 = ld_v4_policy(qs + off + 16 * H, stream);
     const uint32_t w[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
     const float4* g4 = reinterpret_cast<const float4*>(gamma + bj * 32 + c0);
     const float4* b4 = reinterpret_cast<const float4*>(beta + bj * 32 + c0);
@@ -363,8 +364,8 @@ __global__ void __launch_bounds__(kLnThreads, 2) layernorm_i8_kernel(const int8_
     uint32_t o[8];
     quant_pack<32>(v, bq, o);
     int8_t* dst = qo + strip * 32 * H + off;
-    *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
-    *reinterpret_cast<uint4*>(dst + 16 * H) = make_uint4(o[4], o[5], o[6], o[7]);
+    st_v4_policy(dst, make_uint4(o[0], o[1], o[2], o[3]), stream);
+    st_v4_policy(dst + 16 * H, make_uint4(o[4], o[5], o[6], o[7]), stream);
     if (lane == 0) so[strip * nbc + bj] = bq.s;
   }
 }
