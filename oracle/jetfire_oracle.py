@@ -44,7 +44,8 @@ __all__ = [
     "BLOCK", "QMAX", "bf16_bits_to_f32", "f32_to_bf16_bits", "quantize", "quantize_block",
     "dequantize_block", "dequantize", "block_scale_grid", "linear_fwd", "linear_fwd_gelu", "linear_dgrad", "linear_wgrad",
     "requantize", "gelu_i8", "layernorm_i8", "gelu_f64", "quantization_mse", "gelu_grad_f64",
-    "gelu_i8_bwd", "layernorm_i8_bwd",
+    "gelu_i8_bwd", "layernorm_i8_bwd", "E4M3_MAX", "e4m3_encode", "e4m3_decode", "mx_quantize",
+    "mx_dequantize", "mx_linear_fwd",
 ]
 
 
@@ -319,6 +320,57 @@ def layernorm_i8_bwd(xq: np.ndarray, xs: np.ndarray, dyq: np.ndarray, dys: np.nd
     dx32 = dx.astype(np.float32)
     q, s = quantize_block(dx32)
     return q, s, dx32, (dy * xhat).sum(axis=0).astype(np.float32), dy.sum(axis=0).astype(np.float32)
+
+
+# --------------------------------------------------------------------------------------------
+# f4: MXFP8 comparison (not on the path: the B200's hardware block scaling, for a side-by-side
+#     measurement against the per-block INT8 GEMM). OCP Microscaling Formats (MX) v1.0: blocks of
+#     32 consecutive elements along the contraction axis share one E8M0 scale X = 2^e with
+#     e = floor(log2(max |x|)) - emax (emax = 8 for E4M3); elements x / X are converted to E4M3.
+# --------------------------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def e4m3_encode(v: np.ndarray) -> np.ndarray:
+    """fp32 -> FP8 E4M3 bit patterns: round to nearest, ties to even, saturating to +-448."""
+    import torch
+    v = np.clip(np.asarray(v, np.float32), -E4M3_MAX, E4M3_MAX)
+    return torch.from_numpy(np.ascontiguousarray(v)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """FP8 E4M3 bit patterns -> exact fp32 values."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(codes, np.uint8)).view(torch.float8_e4m3fn).to(torch.float32).numpy()
+
+
+def mx_quantize(x: np.ndarray):
+    """MXFP8 (E4M3 elements, E8M0 scales) along the last axis of x [R, K] (K a multiple of 32).
+    Per 1x32 block: e = floor(log2(max |x|)) - 8, clamped to [-127, 127] (an all-zero block takes
+    -127); elements x * 2^-e (exact) rounded to E4M3, ties to even, saturating at +-448 (values in
+    [448, 512) * 2^e are clamped, as the format's rule allows). Returns (codes uint8 [R, K],
+    scale bytes uint8 [R, K/32] holding e + 127)."""
+    x = np.asarray(x, np.float32)
+    R, K = x.shape
+    xb = x.reshape(R, K // 32, 32)
+    amax = np.abs(xb).max(axis=2)
+    _, ex = np.frexp(amax)                               # amax = m 2^ex, m in [0.5, 1)
+    e = np.where(amax > 0, ex - 1 - 8, -127).clip(-127, 127).astype(np.int64)
+    scaled = np.ldexp(xb.astype(np.float64), -e[..., None]).astype(np.float32)  # exact: a power of two
+    return e4m3_encode(scaled).reshape(R, K), (e + 127).astype(np.uint8)
+
+
+def mx_dequantize(codes: np.ndarray, sbytes: np.ndarray) -> np.ndarray:
+    """Exact values (fp64) of an MXFP8 tensor: E4M3 value times 2^(byte - 127)."""
+    v = e4m3_decode(codes).astype(np.float64)
+    R, K = v.shape
+    return np.ldexp(v.reshape(R, K // 32, 32), (sbytes.astype(np.int64) - 127)[..., None]).reshape(R, K)
+
+
+def mx_linear_fwd(Aq, As, Bq, Bs):
+    """Y = A B^T for MXFP8 A [M, K], B [N, K]: every product of two E4M3 values and every power-of-two
+    scale is exact in fp64, and so are the per-block sums; the fp64 total is rounded once to fp32."""
+    return (mx_dequantize(Aq, As) @ mx_dequantize(Bq, Bs).T).astype(np.float32)
 
 
 def quantization_mse(x: np.ndarray, granularity: str) -> float:

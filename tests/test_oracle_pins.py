@@ -532,3 +532,77 @@ def test_granularity_variants_relations_and_bounds():
     # dequantize at any granularity is fp32(q) * s of the element's group
     y = O.dequantize(qt, st, 1, C)
     assert np.array_equal(y, (qt.astype(np.float32) * st.astype(np.float32)).astype(np.float32))
+
+
+# ---------------------------------------------------------------------------------------------
+# f4: MXFP8 comparison
+# ---------------------------------------------------------------------------------------------
+def _e4m3_values():
+    """All finite E4M3 values from the format's definition (1 sign, 4 exponent bits with bias 7,
+    3 mantissa bits; exponent field 0 is subnormal; 0x7F / 0xFF are NaN)."""
+    vals = {}
+    for c in range(256):
+        sgn = -1.0 if c & 0x80 else 1.0
+        ef, mf = (c >> 3) & 0xF, c & 0x7
+        if ef == 0xF and mf == 0x7:
+            continue
+        vals[c] = sgn * (mf / 8.0 * 2.0 ** -6 if ef == 0 else (1 + mf / 8.0) * 2.0 ** (ef - 7))
+    return vals
+
+
+def test_e4m3_encode_is_nearest_even_with_saturation():
+    vals = _e4m3_values()
+    pos = sorted({v for v in vals.values() if v >= 0})
+    rng = np.random.default_rng(50)
+    xs = np.concatenate([rng.normal(0, 30, 3000), rng.uniform(-500, 500, 1000),
+                         [(a + b) / 2 for a, b in zip(pos[:-1], pos[1:])],          # every tie
+                         [-(a + b) / 2 for a, b in zip(pos[:-1], pos[1:])], [448.0, 460.0, 1e6, -1e6, 0.0]])
+    xs = xs.astype(np.float32)
+    codes = O.e4m3_encode(xs)
+    dec = O.e4m3_decode(codes)
+    for x, c, d in zip(xs, codes, dec):
+        a = min(abs(float(x)), 448.0)
+        best = min(pos, key=lambda p: (abs(p - a), [k for k, v in vals.items() if v == p and k < 128][0] & 1))
+        assert abs(float(d)) == best, (x, d, best)
+        assert d == 0 or np.sign(d) == np.sign(x)
+    assert vals[int(O.e4m3_encode(np.array([448.0], np.float32))[0])] == 448.0
+
+
+def test_mx_quantize_rule_hand_and_bounds():
+    # one block 1..32: amax 32 -> e = 5 - 8 = -3, elements x * 8 = 8..256; E4M3 keeps 4 significant
+    # bits, so 17 * 8 = 136 (between 128 and 144, a tie) goes to 128 and 18 * 8 = 144 stays
+    x = np.arange(1, 33, dtype=np.float32)[None, :]
+    q, sb = O.mx_quantize(x)
+    assert sb[0, 0] == 127 - 3
+    y = O.mx_dequantize(q, sb)[0]
+    assert y[0] == 1.0 and y[16] == 16.0 and y[17] == 18.0 and y[31] == 32.0
+    assert O.e4m3_decode(q)[0, 16] == 128.0          # 17 * 8 = 136 -> 128 (tie to even)
+    # random blocks: the block max decodes to [256, 448] x 2^e, elements within half an E4M3 ulp
+    rng = np.random.default_rng(51)
+    x = S.activation(rng, 64, 256, 3, 30.0)
+    x[0, :32] = 0.0
+    q, sb = O.mx_quantize(x)
+    assert sb[0, 0] == 0                              # all-zero block: e = -127
+    v = O.e4m3_decode(q).astype(np.float64).reshape(64, 8, 32)
+    e = sb.astype(np.int64) - 127
+    nz = np.abs(x.reshape(64, 8, 32)).max(axis=2) > 0
+    vmax = np.abs(v).max(axis=2)
+    assert np.all((vmax[nz] >= 256) & (vmax[nz] <= 448))
+    scaled = np.ldexp(x.reshape(64, 8, 32).astype(np.float64), -e[..., None])
+    ulp = np.ldexp(1.0, np.floor(np.log2(np.maximum(np.abs(scaled), 2.0 ** -6))).astype(int) - 3)
+    err = np.abs(np.clip(scaled, -448, 448) - v)
+    assert np.all(err <= ulp / 2 + 1e-12)
+
+
+def test_mx_linear_fwd_exact_small_integers():
+    """Codes that decode to small integers and power-of-two scales: the oracle's Y equals the int64
+    product times the scales exactly, and the modes of the MX GEMM compose like the INT8 one."""
+    rng = np.random.default_rng(52)
+    M, N, K = 64, 96, 256
+    ints = lambda r, c: rng.integers(-15, 16, size=(r, c)).astype(np.float32)
+    A, B = ints(M, K), ints(N, K)
+    Aq, As = O.e4m3_encode(A), np.full((M, K // 32), 127 + 2, np.uint8)     # scale 2^2
+    Bq, Bs = O.e4m3_encode(B), np.full((N, K // 32), 127 - 1, np.uint8)     # scale 2^-1
+    assert np.array_equal(O.e4m3_decode(Aq), A) and np.array_equal(O.e4m3_decode(Bq), B)
+    y = O.mx_linear_fwd(Aq, As, Bq, Bs)
+    assert np.array_equal(y.astype(np.float64), (A.astype(np.int64) @ B.astype(np.int64).T) * 2.0)
