@@ -54,7 +54,7 @@ def parse_args():
     p.add_argument("--sweep-m", type=int, nargs="*", default=[1024, 8192, 65536])
     p.add_argument("--sweep-ops", nargs="*", default=["quantize_bf16", "dequantize_bf16", "gelu_i8", "layernorm_i8",
                                                       "gelu_i8_bwd", "layernorm_i8_bwd", "fused_fc1",
-                                                      "granularity_mse"])
+                                                      "granularity_mse", "mxfp8_fc1"])
     return p.parse_args()
 
 
@@ -591,9 +591,55 @@ def run_sweep(args):
         out.update(_sweep_fused_fc1(jf, flush))
     if "granularity_mse" in args.sweep_ops:
         out["granularity_mse"] = _granularity_mse(jf)
+    if "mxfp8_fc1" in args.sweep_ops:
+        out["mxfp8_vs_int8_fc1"] = _mxfp8_vs_int8(jf, flush)
     assert jf.jf_device_status() == 0
     print(json.dumps({"sweep": out, "hbm_peak_gbs": peaks["hbm_gbs"], "peak_source": peak_src,
                       "l2": "flushed before every timed launch"}), flush=True)
+
+
+def _mxfp8_vs_int8(jf, flush):
+    """The GPT2-medium fc1 forward (M=4096, K=1024, N=4096, bf16 inputs) two ways: Jetfire's 32x32
+    INT8 blocks (quantize X and W, block-scaled INT8 GEMM with fp32 output) and MXFP8 (1x32 E8M0
+    blocks, E4M3 elements, the tensor core's block-scaled MMA). Device times (L2 flushed before each
+    launch) and the relative Frobenius error of each fp32 output against the exact product of the
+    bf16 inputs (fp64 on the host)."""
+    import torch
+    wl = __import__("inputs.synthetic", fromlist=["WORKLOADS"]).WORKLOADS[WORKLOAD]
+    M, K, N = wl["M"], wl["K"], wl["N"]
+    host = host_inputs(M, K, N, 0, seed_weight=0)
+    xb = torch.from_numpy(host["x"].view(np.int16)).cuda().view(torch.bfloat16)
+    wb = torch.from_numpy(host["w"].view(np.int16)).cuda().view(torch.bfloat16)
+    ref = (xb.cpu().double().numpy() @ wb.cpu().double().numpy().T)
+
+    def timed(fn, reps=10):
+        for _ in range(3):
+            flush.zero_()
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(); fn(); b.record()
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in ts)
+
+    res = {}
+    X, W = jf.quantize_block(xb), jf.quantize_block(wb)
+    Y, yf = jf.empty_qtensor(M, N), torch.empty((M, N), dtype=torch.float32, device="cuda")
+    q_ms = timed(lambda: (jf.jf_quantize_block(xb, X.q, X.s), jf.jf_quantize_block(wb, W.q, W.s)))
+    g_ms = timed(lambda: jf.jf_linear_fwd(X, W, None, yf))
+    err = float(np.linalg.norm(yf.cpu().double().numpy() - ref) / np.linalg.norm(ref))
+    res["int8_32x32"] = {"quantize_ms": round(q_ms, 4), "gemm_ms": round(g_ms, 4),
+                         "gemm_TOPS": round(2 * M * N * K / (g_ms * 1e-3) / 1e12, 1), "rel_error": float(f"{err:.4g}")}
+    (Aq, As), (Bq, Bs) = jf.mx_quantize(xb), jf.mx_quantize(wb)
+    q_ms = timed(lambda: (jf.jf_mx_quantize(xb, Aq, As), jf.jf_mx_quantize(wb, Bq, Bs)))
+    g_ms = timed(lambda: jf.jf_mx_linear_fwd(Aq, As, Bq, Bs, yf))
+    err = float(np.linalg.norm(yf.cpu().double().numpy() - ref) / np.linalg.norm(ref))
+    res["mxfp8_1x32"] = {"quantize_ms": round(q_ms, 4), "gemm_ms": round(g_ms, 4),
+                         "gemm_TOPS": round(2 * M * N * K / (g_ms * 1e-3) / 1e12, 1), "rel_error": float(f"{err:.4g}")}
+    return res
 
 
 def _granularity_mse(jf):

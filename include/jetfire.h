@@ -235,6 +235,26 @@ JF_API int jf_dequantize_granular(const int8_t* q, const float* s, int64_t rows,
 JF_API int jf_quantization_error(const void* x, jf_dtype dt, const int8_t* q, const float* s, int64_t rows,
                                  int64_t cols, jf_granularity g, double* sums, void* stream);
 
+/*
+ * f4. MXFP8 comparison (OCP Microscaling Formats v1.0; not on the pages: the B200's hardware block
+ *     scaling, measured beside the per-block INT8 path). Quantization of x [rows, cols] (dtype dt,
+ *     16-byte aligned) in blocks of 32 consecutive elements of a row: e = floor(log2(max |x|)) - 8
+ *     clamped to [-127, 127] (-127 for an all-zero block), scale byte e + 127 (E8M0), codes = E4M3
+ *     of x * 2^-e, round to nearest even, saturating at +-448.
+ *   codes   uint8 [rows, cols], 16-byte aligned; scales uint8 [rows, cols / 32]. Bit-exact.
+ */
+JF_API int jf_mx_quantize(const void* x, jf_dtype dt, int64_t rows, int64_t cols, uint8_t* codes, uint8_t* scales,
+                          void* stream);
+
+/*
+ * f4. Y = A B^T with A [M, K] and B [N, K] in MXFP8 (codes and scale bytes as jf_mx_quantize
+ *     writes them), on tcgen05.mma kind::mxf8f6f4.block_scale: the tensor core applies the scales
+ *     and accumulates in fp32. y fp32 [M, N] (16-byte aligned). K must be a positive multiple of 128
+ *     and the scale arrays 4-byte aligned (JF_ERR_SHAPE / JF_ERR_ALIGN otherwise).
+ */
+JF_API int jf_mx_linear_fwd(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
+                            const uint8_t* b_scales, int64_t M, int64_t N, int64_t K, float* y, void* stream);
+
 /* Static description of a status code (never NULL). */
 JF_API const char* jf_strerror(int status);
 

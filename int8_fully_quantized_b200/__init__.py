@@ -28,11 +28,13 @@ __all__ = [
     "jf_quantize_block", "jf_dequantize_block", "jf_linear_fwd", "jf_linear_fwd_gelu", "jf_linear_dgrad",
     "jf_linear_wgrad", "jf_gelu_i8", "jf_layernorm_i8", "jf_gelu_i8_bwd", "jf_layernorm_i8_bwd",
     "jf_layernorm_i8_bwd_workspace_bytes", "jf_layernorm_i8_bwd_noalloc", "jf_quantize_granular",
-    "jf_dequantize_granular", "jf_quantization_error", "jf_granular_scale_count", "jf_strerror",
+    "jf_dequantize_granular", "jf_quantization_error", "jf_granular_scale_count", "jf_mx_quantize",
+    "jf_mx_linear_fwd", "jf_strerror",
     "jf_device_status", "jf_sm_count",
     # allocating helpers
     "quantize_block", "dequantize_block", "linear_fwd", "linear_fwd_gelu", "linear_dgrad", "linear_wgrad",
     "gelu_i8", "layernorm_i8", "gelu_i8_bwd", "layernorm_i8_bwd", "quantize_granular", "quantization_mse",
+    "mx_quantize", "mx_linear_fwd",
 ]
 
 JF_F32, JF_BF16, JF_F16 = 0, 1, 2
@@ -44,7 +46,8 @@ EXPORTED_SYMBOLS = (
     "jf_linear_wgrad",
     "jf_gelu_i8", "jf_layernorm_i8", "jf_gelu_i8_bwd", "jf_layernorm_i8_bwd", "jf_layernorm_i8_bwd_workspace_bytes",
     "jf_layernorm_i8_bwd_noalloc", "jf_quantize_granular", "jf_dequantize_granular", "jf_quantization_error",
-    "jf_granular_scale_count", "jf_strerror", "jf_device_status", "jf_sm_count",
+    "jf_granular_scale_count", "jf_mx_quantize", "jf_mx_linear_fwd", "jf_strerror", "jf_device_status",
+    "jf_sm_count",
 )
 
 
@@ -93,6 +96,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.jf_dequantize_granular.argtypes = [vp, vp, i64, i64, i32, vp, i32, vp]
     lib.jf_quantization_error.argtypes = [vp, i32, vp, vp, i64, i64, i32, vp, vp]
     lib.jf_granular_scale_count.argtypes = [i64, i64, i32]
+    lib.jf_mx_quantize.argtypes = [vp, i32, i64, i64, vp, vp, vp]
+    lib.jf_mx_linear_fwd.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp]
     lib.jf_strerror.argtypes = [i32]
     lib.jf_strerror.restype = ctypes.c_char_p
     lib.jf_device_status.argtypes = [vp]
@@ -273,6 +278,35 @@ def quantization_mse(x: torch.Tensor, granularity: str, stream=None) -> float:
     sums = torch.empty(2, dtype=torch.float64, device=x.device)
     jf_quantization_error(x, q, s, GRANULARITY[granularity], sums, stream)
     return float(sums[0].item()) / x.numel()
+
+
+def jf_mx_quantize(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, stream=None) -> None:
+    lib = load_library()
+    _check(lib.jf_mx_quantize(_ptr(x), _DTYPES[x.dtype], x.shape[0], x.shape[1], _ptr(codes), _ptr(scales),
+                              _stream(stream)), "jf_mx_quantize")
+
+
+def jf_mx_linear_fwd(a_codes, a_scales, b_codes, b_scales, y: torch.Tensor, stream=None) -> None:
+    lib = load_library()
+    M, K = a_codes.shape
+    N = b_codes.shape[0]
+    _check(lib.jf_mx_linear_fwd(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), M, N, K, _ptr(y),
+                                _stream(stream)), "jf_mx_linear_fwd")
+
+
+def mx_quantize(x: torch.Tensor, stream=None):
+    """MXFP8 (E4M3 codes as uint8, E8M0 scale bytes per 1x32 block of a row) of x [rows, cols]."""
+    codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    scales = torch.empty((x.shape[0], x.shape[1] // 32), dtype=torch.uint8, device=x.device)
+    jf_mx_quantize(x, codes, scales, stream)
+    return codes, scales
+
+
+def mx_linear_fwd(a_codes, a_scales, b_codes, b_scales, stream=None) -> torch.Tensor:
+    """fp32 Y = A B^T of two MXFP8 tensors on the tensor core's block-scaled MMA."""
+    y = torch.empty((a_codes.shape[0], b_codes.shape[0]), dtype=torch.float32, device=a_codes.device)
+    jf_mx_linear_fwd(a_codes, a_scales, b_codes, b_scales, y, stream)
+    return y
 
 
 def jf_strerror(status: int) -> str:

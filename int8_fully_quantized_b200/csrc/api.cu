@@ -386,6 +386,41 @@ int jf_quantization_error(const void* x, jf_dtype dt, const int8_t* q, const flo
                                             static_cast<cudaStream_t>(stream)));
 }
 
+int jf_mx_quantize(const void* x, jf_dtype dt, int64_t rows, int64_t cols, uint8_t* codes, uint8_t* scales,
+                   void* stream) {
+  if (dt != JF_F32 && dt != JF_BF16 && dt != JF_F16) return JF_ERR_DTYPE;
+  if (!dims_ok(rows, cols)) return JF_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return JF_OK;
+  if (x == nullptr || codes == nullptr || scales == nullptr) return JF_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(codes, 16)) return JF_ERR_ALIGN;
+  const int64_t nx = rows * cols * elem_size(dt), nc = rows * cols, ns = rows * (cols / 32);
+  if (overlap(codes, nc, x, nx) || overlap(scales, ns, x, nx) || overlap(codes, nc, scales, ns)) return JF_ERR_ALIAS;
+  const DevInfo d = device_info();
+  if (!d.ok) return JF_ERR_DEVICE;
+  return cuda_status(jf::launch_mx_quantize(x, int(dt), rows, cols, codes, scales, d.sm_count,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+int jf_mx_linear_fwd(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes, const uint8_t* b_scales,
+                     int64_t M, int64_t N, int64_t K, float* y, void* stream) {
+  if (!dims_ok(M, K) || !dims_ok(N, K) || K % 128 != 0) return JF_ERR_SHAPE;
+  if (M == 0 || N == 0) return JF_OK;
+  if (K == 0) return JF_ERR_SHAPE;
+  if (a_codes == nullptr || a_scales == nullptr || b_codes == nullptr || b_scales == nullptr || y == nullptr)
+    return JF_ERR_NULL;
+  if (!aligned(a_codes, 16) || !aligned(b_codes, 16) || !aligned(a_scales, 4) || !aligned(b_scales, 4) ||
+      !aligned(y, 16))
+    return JF_ERR_ALIGN;
+  const void* ins[4] = {a_codes, a_scales, b_codes, b_scales};
+  const int64_t in_n[4] = {M * K, M * (K / 32), N * K, N * (K / 32)};
+  for (int i = 0; i < 4; ++i)
+    if (overlap(y, M * N * 4, ins[i], in_n[i])) return JF_ERR_ALIAS;
+  const DevInfo d = device_info();
+  if (!d.ok) return JF_ERR_DEVICE;
+  return cuda_status(jf::launch_mx_gemm(a_codes, a_scales, b_codes, b_scales, M, N, K, y, d.status, d.sm_count,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 const char* jf_strerror(int status) {
   switch (status) {
     case JF_OK: return "ok";

@@ -95,11 +95,6 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
          (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (uint64_t(1) << 46) | (uint64_t(2) << 61);
 }
 
-// Bounded wait for teardown: ignores the abort flag, still gives up after the watchdog time.
-__device__ __forceinline__ void mbar_wait_teardown(uint64_t* bar, uint32_t parity, unsigned int* status) {
-  uint32_t dummy = 0;
-  mbar_wait(bar, parity, &dummy, status);
-}
 
 // Re-quantize one warp's 32x32 fp32 block (lane = row; the row's 32 values in acc) and store its
 // codes at q (lane's row, ld_y-strided by the caller's offset) and its scale at *s.

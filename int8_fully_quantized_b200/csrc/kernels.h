@@ -12,6 +12,13 @@ cudaError_t launch_dequantize(const int8_t* q, const float* s, int64_t R, int64_
                               int sm_count, cudaStream_t st);
 cudaError_t launch_gelu_i8(const int8_t* q, const float* s, int64_t R, int64_t C, int8_t* qo, float* so,
                            int sm_count, cudaStream_t st);
+// MXFP8 comparison path (mxfp8.cu): MX quantization (E4M3 codes, E8M0 scale bytes per 1x32 block of
+// a row) and Y = A B^T with the tensor core's block scaling (K a multiple of 128).
+cudaError_t launch_mx_quantize(const void* x, int dtype, int64_t R, int64_t K, uint8_t* codes, uint8_t* scales,
+                               int sm_count, cudaStream_t st);
+cudaError_t launch_mx_gemm(const uint8_t* a_q, const uint8_t* a_s, const uint8_t* b_q, const uint8_t* b_s, int64_t M,
+                           int64_t N, int64_t K, float* y, unsigned int* status, int sm_count, cudaStream_t st);
+
 // Granularity variants of the quantizer and the quantization-error sums (granular.cu). Scales:
 // block [R/32, C/32], token [R], channel [C], tensor [1].
 enum Granularity { kGranBlock = 0, kGranToken = 1, kGranChannel = 2, kGranTensor = 3 };
