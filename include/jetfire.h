@@ -255,6 +255,14 @@ JF_API int jf_mx_quantize(const void* x, jf_dtype dt, int64_t rows, int64_t cols
 JF_API int jf_mx_linear_fwd(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
                             const uint8_t* b_scales, int64_t M, int64_t N, int64_t K, float* y, void* stream);
 
+/*
+ * Self-test of the failure path (no counterpart on the pages): enqueues a kernel whose bounded wait
+ * on a barrier that nothing arrives on gives up after limit_ns nanoseconds (1 ms .. 10 s, else
+ * JF_ERR_ARG), the same way any kernel of the library gives up a wait. The next jf_device_status
+ * then returns JF_ERR_TIMEOUT and clears the status; the context stays usable.
+ */
+JF_API int jf_selftest_wait_timeout(int64_t limit_ns, void* stream);
+
 /* Static description of a status code (never NULL). */
 JF_API const char* jf_strerror(int status);
 

@@ -29,7 +29,7 @@ __all__ = [
     "jf_linear_wgrad", "jf_gelu_i8", "jf_layernorm_i8", "jf_gelu_i8_bwd", "jf_layernorm_i8_bwd",
     "jf_layernorm_i8_bwd_workspace_bytes", "jf_layernorm_i8_bwd_noalloc", "jf_quantize_granular",
     "jf_dequantize_granular", "jf_quantization_error", "jf_granular_scale_count", "jf_mx_quantize",
-    "jf_mx_linear_fwd", "jf_strerror",
+    "jf_mx_linear_fwd", "jf_selftest_wait_timeout", "jf_strerror",
     "jf_device_status", "jf_sm_count",
     # allocating helpers
     "quantize_block", "dequantize_block", "linear_fwd", "linear_fwd_gelu", "linear_dgrad", "linear_wgrad",
@@ -46,7 +46,8 @@ EXPORTED_SYMBOLS = (
     "jf_linear_wgrad",
     "jf_gelu_i8", "jf_layernorm_i8", "jf_gelu_i8_bwd", "jf_layernorm_i8_bwd", "jf_layernorm_i8_bwd_workspace_bytes",
     "jf_layernorm_i8_bwd_noalloc", "jf_quantize_granular", "jf_dequantize_granular", "jf_quantization_error",
-    "jf_granular_scale_count", "jf_mx_quantize", "jf_mx_linear_fwd", "jf_strerror", "jf_device_status",
+    "jf_granular_scale_count", "jf_mx_quantize", "jf_mx_linear_fwd", "jf_selftest_wait_timeout", "jf_strerror",
+    "jf_device_status",
     "jf_sm_count",
 )
 
@@ -98,6 +99,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.jf_granular_scale_count.argtypes = [i64, i64, i32]
     lib.jf_mx_quantize.argtypes = [vp, i32, i64, i64, vp, vp, vp]
     lib.jf_mx_linear_fwd.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp]
+    lib.jf_selftest_wait_timeout.argtypes = [i64, vp]
     lib.jf_strerror.argtypes = [i32]
     lib.jf_strerror.restype = ctypes.c_char_p
     lib.jf_device_status.argtypes = [vp]
@@ -307,6 +309,11 @@ def mx_linear_fwd(a_codes, a_scales, b_codes, b_scales, stream=None) -> torch.Te
     y = torch.empty((a_codes.shape[0], b_codes.shape[0]), dtype=torch.float32, device=a_codes.device)
     jf_mx_linear_fwd(a_codes, a_scales, b_codes, b_scales, y, stream)
     return y
+
+
+def jf_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    lib = load_library()
+    _check(lib.jf_selftest_wait_timeout(limit_ns, _stream(stream)), "jf_selftest_wait_timeout")
 
 
 def jf_strerror(status: int) -> str:

@@ -421,6 +421,14 @@ int jf_mx_linear_fwd(const uint8_t* a_codes, const uint8_t* a_scales, const uint
                                         static_cast<cudaStream_t>(stream)));
 }
 
+int jf_selftest_wait_timeout(int64_t limit_ns, void* stream) {
+  if (limit_ns < 1000000 || limit_ns > 10000000000ll) return JF_ERR_ARG;
+  const DevInfo d = device_info();
+  if (!d.ok) return JF_ERR_DEVICE;
+  return cuda_status(jf::launch_wait_selftest(d.status, static_cast<unsigned long long>(limit_ns),
+                                              static_cast<cudaStream_t>(stream)));
+}
+
 const char* jf_strerror(int status) {
   switch (status) {
     case JF_OK: return "ok";

@@ -12,6 +12,10 @@ cudaError_t launch_dequantize(const int8_t* q, const float* s, int64_t R, int64_
                               int sm_count, cudaStream_t st);
 cudaError_t launch_gelu_i8(const int8_t* q, const float* s, int64_t R, int64_t C, int8_t* qo, float* so,
                            int sm_count, cudaStream_t st);
+// Failure-path self-test (selftest.cu): a bounded wait that runs out after limit_ns and raises the
+// timeout bit of *status.
+cudaError_t launch_wait_selftest(unsigned int* status, unsigned long long limit_ns, cudaStream_t st);
+
 // MXFP8 comparison path (mxfp8.cu): MX quantization (E4M3 codes, E8M0 scale bytes per 1x32 block of
 // a row) and Y = A B^T with the tensor core's block scaling (K a multiple of 128).
 cudaError_t launch_mx_quantize(const void* x, int dtype, int64_t R, int64_t K, uint8_t* codes, uint8_t* scales,

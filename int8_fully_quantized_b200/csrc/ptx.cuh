@@ -54,14 +54,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // becomes nonzero (another thread gave up) or after kWatchdogNs, in which case it raises the
 // timeout bit of *status, sets *abort and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort,
-                                          unsigned int* status) {
+                                          unsigned int* status, unsigned long long limit_ns = kWatchdogNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((n & 63u) == 0) {
       if (*abort) return false;
-      if (globaltimer() - t0 > kWatchdogNs) {
+      if (globaltimer() - t0 > limit_ns) {
         *abort = 1u;
         atomicOr(status, kStatusTimeout);
         return false;
