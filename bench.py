@@ -199,13 +199,14 @@ class GpuStep:
         }
         self.ops = {"linear_fwd": 2 * M * N * K, "linear_dgrad": 2 * M * K * N, "linear_wgrad": 2 * N * K * M}
         self.side = torch.cuda.Stream(device=dev)
-        self.w_ready = torch.cuda.Event()
+        self.w_ready, self.dy_ready, self.xn_ready = torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event()
         self.graph = None
 
     def run_overlapped(self):
-        """The same nine operators, with the two that depend on neither X nor each other (quantize W,
-        quantize dY) on a second stream, overlapping quantize X and LayerNorm_i8; the forward waits
-        for W, the backward for dY."""
+        """The same nine operators on two streams, ordered by their data dependences only: quantize W
+        and quantize dY run beside quantize X and LayerNorm_i8, and the weight gradient (dY^T Xn)
+        needs neither the forward nor GELU, so it runs beside them and the input gradient; the
+        persistent GEMMs then fill each other's last partial wave of tiles."""
         jf, t = self.jf, self.torch
         main = t.cuda.current_stream()
         self.side.wait_stream(main)
@@ -213,15 +214,20 @@ class GpuStep:
             jf.jf_quantize_block(self.wb, self.Wq.q, self.Wq.s)
             self.w_ready.record()
             jf.jf_quantize_block(self.dyb, self.dYq.q, self.dYq.s)
+            self.dy_ready.record()
         jf.jf_quantize_block(self.xb, self.Xq.q, self.Xq.s)
         jf.jf_layernorm_i8(self.Xq, self.gamma, self.beta, 1e-5, self.Xn)
+        self.xn_ready.record()
+        with t.cuda.stream(self.side):
+            self.side.wait_event(self.xn_ready)
+            jf.jf_linear_wgrad(self.dYq, self.Xn, self.dW, None)
         main.wait_event(self.w_ready)
         jf.jf_linear_fwd(self.Xn, self.Wq, self.Y, None)
         jf.jf_gelu_i8(self.Y, self.G)
-        main.wait_stream(self.side)
+        main.wait_event(self.dy_ready)
         jf.jf_linear_dgrad(self.dYq, self.Wq, self.dX, None)
-        jf.jf_linear_wgrad(self.dYq, self.Xn, self.dW, None)
         jf.jf_dequantize_block(self.dX.q, self.dX.s, self.dx_bf16)
+        main.wait_stream(self.side)
 
     def capture(self):
         """CUDA graph of run_overlapped (single GPU): one replay launches the step's kernels with no
@@ -380,8 +386,9 @@ def run_ours(args):
                    "inputs": "bf16 X ~N(0,1) with 10 channels x30, W ~N(0,0.02), dY ~N(0,1e-3)",
                    "parallelism": f"dp{world}", "l2": "flushed between steps (256 MiB write, outside timed events)"},
         "kernels": kernels, "roofline": roofline,
-        "execution": ("CUDA graph of the step, quantize W and dY on a second stream overlapping quantize X and "
-                      "LayerNorm_i8; per-kernel times from the nine operators serialized on one stream"
+        "execution": ("CUDA graph of the step on two streams ordered by data dependences (quantize W, quantize dY "
+                      "and the weight gradient beside quantize X, LayerNorm_i8, the forward, GELU_i8 and the input "
+                      "gradient); per-kernel times from the nine operators serialized on one stream"
                       if use_graph else "eager launches on one stream, per-kernel events"),
         "gpu_launches": step.launches_per_step * args.steps,
         "clocks": sampler.summary(),
