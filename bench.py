@@ -48,6 +48,8 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     p.add_argument("--eager", action="store_true", help="time eager launches instead of the step's CUDA graph")
+    p.add_argument("--configs", action="store_true",
+                   help="time the single-linear, hidden-4096 GEMM and hidden-4096 MLP-block workloads (one JSON line)")
     p.add_argument("--cpu-sample-tokens", type=int, default=1024)
     p.add_argument("--sweep", action="store_true",
                    help="time the memory-bound kernels on the M x 4096 sweep instead of the step")
@@ -700,8 +702,117 @@ def _sweep_fused_fc1(jf, flush):
     return res
 
 
+def _device_ms(fn, flush, reps=10):
+    """Median CUDA-event time of fn over reps launches, L2 flushed (256 MiB write) before each."""
+    import torch
+    for _ in range(3):
+        flush.zero_()
+        fn()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(); fn(); b.record()
+        ts.append((a, b))
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in ts)
+
+
+def run_configs(args):
+    """The workloads besides the headline step, each timed on the device (L2 flushed before every
+    launch) with the CPU oracle beside it on the same inputs (whole where it finishes in seconds,
+    else a stated sample):
+      single_linear_256: quantize X and W (fp32 256x256) and the forward, a latency case;
+      h4096_fc1 / h4096_fc2: forward, input- and weight-gradient GEMMs of the hidden-4096 layer;
+      h4096_mlp_block: LayerNorm_i8 -> fc1 -> GELU_i8 -> fc2 on INT8 blocks (M = 8192), and the
+      same with GELU fused into fc1's epilogue."""
+    import torch
+    import int8_fully_quantized_b200 as jf
+    import oracle as O
+    from inputs import synthetic as S
+    torch.cuda.set_device(0)
+    jf.load_library()
+    peaks, peak_src = load_peaks()
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    alu_peak = ALU_LANES_PER_CLK_PER_SM * B200_SMS * peaks["sm_max_mhz"] * 1e6
+    i8_peak = peaks["bf16_tflops"] * NOMINAL_I8_OVER_BF16
+    out = {}
+    # ---- single linear, 256^3, fp32 inputs
+    d = S.workload("linear_256", 0)
+    x, w = torch.from_numpy(d["X"]).cuda(), torch.from_numpy(d["W"]).cuda()
+    X, W, Y = jf.empty_qtensor(256, 256), jf.empty_qtensor(256, 256), jf.empty_qtensor(256, 256)
+    ms = _device_ms(lambda: (jf.jf_quantize_block(x, X.q, X.s), jf.jf_quantize_block(w, W.q, W.s),
+                             jf.jf_linear_fwd(X, W, Y)), flush, reps=20)
+    t0 = time.perf_counter()
+    xq, xs = O.quantize_block(d["X"]); wq, ws = O.quantize_block(d["W"])
+    O.requantize(O.linear_fwd(xq, xs, wq, ws))
+    cpu_s = time.perf_counter() - t0
+    out["single_linear_256"] = {"device_us": round(ms * 1e3, 2), "oracle_ms": round(cpu_s * 1e3, 2),
+                                "note": "three launches (quantize X, quantize W, forward); latency-bound"}
+    del x, w, X, W, Y
+    # ---- hidden-4096 GEMMs
+    for name in ("h4096_fc1", "h4096_fc2"):
+        wl = S.WORKLOADS[name]
+        M, K, N = wl["M"], wl["K"], wl["N"]
+        g = torch.Generator(device="cuda").manual_seed(0)
+        qt = lambda r, c: jf.QTensor(torch.randint(-127, 128, (r, c), dtype=torch.int8, device="cuda", generator=g),
+                                     torch.rand((r // 32, c // 32), device="cuda", generator=g) * 0.01 + 1e-3)
+        A, B, dY = qt(M, K), qt(N, K), qt(M, N)
+        res = {}
+        for mode, fn, rows, cols in (("fwd", lambda o: jf.jf_linear_fwd(A, B, o), M, N),
+                                     ("dgrad", lambda o: jf.jf_linear_dgrad(dY, B, o), M, K),
+                                     ("wgrad", lambda o: jf.jf_linear_wgrad(dY, A, o), N, K)):
+            o = jf.empty_qtensor(rows, cols)
+            ms = _device_ms(lambda: fn(o), flush, reps=5)
+            ops = 2 * M * N * K
+            res[mode] = {"ms": round(ms, 3), "TOPS": round(ops / (ms * 1e-3) / 1e12, 1),
+                         "alu_frac": round(ops / 32 / (ms * 1e-3) / alu_peak, 4),
+                         "tensor_frac": round(ops / (ms * 1e-3) / 1e12 / i8_peak, 4)}
+            del o
+        # oracle: one 32x32 output block of the forward, timed, and its cost for the full output
+        Xh, Wh = host_q(A), host_q(B)
+        t0 = time.perf_counter()
+        O.linear_fwd(*Xh, *Wh, [0], [0])
+        blk = time.perf_counter() - t0
+        res["oracle"] = {"one_block_ms": round(blk * 1e3, 2),
+                         "full_fwd_s_extrapolated": round(blk * (M // 32) * (N // 32), 1)}
+        out[name] = res
+        del A, B, dY
+    # ---- hidden-4096 MLP block on INT8 blocks
+    wl1, wl2 = S.WORKLOADS["h4096_fc1"], S.WORKLOADS["h4096_fc2"]
+    M, H, F = wl1["M"], wl1["K"], wl1["N"]
+    rng = np.random.default_rng(0)
+    xin = torch.from_numpy(S.to_bf16_bits(S.activation(rng, M, H, 4, 50.0)).view(np.int16)).cuda().view(torch.bfloat16)
+    Xq = jf.quantize_block(xin)
+    W1 = jf.quantize_block(torch.from_numpy(S.to_bf16_bits(S.weight(rng, F, H)).view(np.int16)).cuda().view(torch.bfloat16))
+    W2 = jf.quantize_block(torch.from_numpy(S.to_bf16_bits(S.weight(rng, H, F)).view(np.int16)).cuda().view(torch.bfloat16))
+    gamma, beta = torch.ones(H, device="cuda"), torch.zeros(H, device="cuda")
+    Xn, Y1, G, Y2 = jf.empty_qtensor(M, H), jf.empty_qtensor(M, F), jf.empty_qtensor(M, F), jf.empty_qtensor(M, H)
+    chain = lambda: (jf.jf_layernorm_i8(Xq, gamma, beta, 1e-5, Xn), jf.jf_linear_fwd(Xn, W1, Y1), jf.jf_gelu_i8(Y1, G),
+                     jf.jf_linear_fwd(G, W2, Y2))
+    fused = lambda: (jf.jf_layernorm_i8(Xq, gamma, beta, 1e-5, Xn), jf.jf_linear_fwd_gelu(Xn, W1, G),
+                     jf.jf_linear_fwd(G, W2, Y2))
+    ops = 2 * M * F * H * 2
+    ms, msf = _device_ms(chain, flush, reps=5), _device_ms(fused, flush, reps=5)
+    out["h4096_mlp_block"] = {"ms": round(ms, 3), "TOPS": round(ops / (ms * 1e-3) / 1e12, 1),
+                              "fused_gelu_ms": round(msf, 3), "fused_gelu_TOPS": round(ops / (msf * 1e-3) / 1e12, 1),
+                              "note": "GEMM int8 ops of fc1 + fc2 over the block's device time"}
+    assert jf.jf_device_status() == 0
+    print(json.dumps({"configs": out, "peaks": {"alu_T_lane_instr_s": round(alu_peak / 1e12, 2),
+                                                 "int8_tops": round(i8_peak, 1), "source": peak_src},
+                      "l2": "flushed before every timed launch", "cpu_threads": _cpu_cores()}), flush=True)
+
+
+def host_q(t):
+    """(codes, scales) of a device QTensor as host numpy arrays."""
+    return t.q.cpu().numpy(), t.s.cpu().numpy()
+
+
 def main():
     args = parse_args()
+    if args.configs:
+        run_configs(args)
+        return
     if args.sweep:
         run_sweep(args)
         return
