@@ -79,8 +79,9 @@ __global__ void __launch_bounds__(32 * kGeluBwdWarps, 3) gelu_i8_bwd_kernel(
 // H columns of a row, rstd = 1 / sqrt(var + eps)), with xhat = (x - mu) rstd and g = dy gamma:
 //   dx = rstd (g - mean(g) - xhat mean(g xhat)),  dgamma = sum_rows dy xhat,  dbeta = sum_rows dy.
 // Persistent CTAs of 8 warps, three per SM, each looping over 32-row strips:
-//   phase 1: warp w reduces rows w, w + 8, w + 16 and w + 24 of the strip, each in one pass: sums of x, x^2, g and g x (chunk partials
-//            of 16 values in fp32, accumulated in fp64). Then mean, rstd, mean(g) and
+//   phase 1: warp w reduces rows w, w + 8, w + 16 and w + 24 of the strip, each in one pass: sums
+//            of x, x^2, g and g x over 16-value chunks (the x sums exact in integers, the g sums in
+//            fp32 before the block scales), scaled and accumulated in fp64. Then mean, rstd, mean(g) and
 //            mean(g xhat) = rstd (mean(g x) - mean * mean(g)) per row, kept in shared memory.
 //   phase 2: warp w handles column blocks w, w + 8, ...: lane l takes the 4 columns 4 (l % 8) .. +3
 //            of rows l / 8 + 4 i (i = 0..7), computes dx, re-quantizes the block and sums dy xhat
@@ -140,7 +141,8 @@ __global__ void __launch_bounds__(kLnbThreads, 3) layernorm_i8_bwd_kernel(
           const uint32_t wx[4] = {av[u].x, av[u].y, av[u].z, av[u].w};
           const uint32_t wd[4] = {dv[u].x, dv[u].y, dv[u].z, dv[u].w};
           const float4* g4 = reinterpret_cast<const float4*>(gamma + ch * 16);
-          float px = 0.0f, pxx = 0.0f, pg = 0.0f, pgx = 0.0f;
+          // the chunk's codes share one block scale per tensor: the scales are applied once per chunk
+          float pg = 0.0f, pgx = 0.0f;  // sums of q_dy gamma and q_dy gamma q_x over the chunk
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const float4 gm = __ldg(g4 + i);
@@ -150,18 +152,16 @@ __global__ void __launch_bounds__(kLnbThreads, 3) layernorm_i8_bwd_kernel(
             i8x4_to_f32(wd[i], fd);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-              const float x = fx[j] * scx[u];
-              const float g = (fd[j] * scd[u]) * gmv[j];
-              px += x;
-              pxx = fmaf(x, x, pxx);
-              pg += g;
-              pgx = fmaf(g, x, pgx);
+              const float t = fd[j] * gmv[j];
+              pg += t;
+              pgx = fmaf(t, fx[j], pgx);
             }
           }
-          sum_x += double(px);
-          sum_xx += double(pxx);
-          sum_g += double(pg);
-          sum_gx += double(pgx);
+          const double sx = double(scx[u]), sd = double(scd[u]);
+          sum_x = fma(sx, double(chunk_sum_i8(av[u])), sum_x);  // exact integer sums of the x codes
+          sum_xx = fma(sx * sx, double(chunk_sumsq_i8(av[u])), sum_xx);
+          sum_g = fma(sd, double(pg), sum_g);
+          sum_gx = fma(sd * sx, double(pgx), sum_gx);
         }
       }
 #pragma unroll

@@ -251,9 +251,10 @@ __global__ void __launch_bounds__(32 * kGeluWarps, 3) gelu_i8_kernel(const int8_
 // ---------------------------------------------------------------------------------------------
 // a7: LayerNorm_i8. One CTA of 16 warps per 32-row strip [32, H]; two CTAs share an SM so that
 // one's reduction overlaps the other's output phase.
-//   phase 1: warp w reduces rows w and w + 16: sum and sum of squares of x = fp32(q) * s (chunk
-//            partials of 16 values in fp32, accumulated in fp64), then mean, biased variance and
-//            rstd = 1 / sqrt(var + eps) in fp64, kept in shared memory.
+//   phase 1: warp w reduces rows w and w + 16: sum and sum of squares of x = q * s, from exact
+//            integer sums of each 16-code chunk (one block scale per chunk) scaled and accumulated
+//            in fp64, then mean, biased variance and rstd = 1 / sqrt(var + eps) in fp64, kept in
+//            shared memory.
 //   phase 2: warp w handles column blocks w, w + 16, ...: y = (x - mean) * rstd * gamma + beta in
 //            fp32, block absmax, per-block re-quantization. The strip is read a second time; it
 //            is at most 32 * H bytes and is still in L2.
@@ -293,23 +294,12 @@ __global__ void __launch_bounds__(kLnThreads, 2) layernorm_i8_kernel(const int8_
       }
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
-      const uint4 a = av[u];
-      const float sc = scv[u];
-      const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-      float ps = 0.0f, pq = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float g[4];
-        i8x4_to_f32(w[i], g);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float x = g[j] * sc;
-          ps += x;
-          pq = fmaf(x, x, pq);
-        }
-      }
-      sum += double(ps);
-      sq += double(pq);
+        // the 16 codes of a chunk share one block scale: their sum and sum of squares are exact
+        // integers (4-way byte dot products), scaled once in fp64
+        const int is = chunk_sum_i8(av[u]), iq = chunk_sumsq_i8(av[u]);
+        const double sc = double(scv[u]);
+        sum = fma(sc, double(is), sum);
+        sq = fma(sc * sc, double(iq), sq);
       }
     }
 #pragma unroll
@@ -337,27 +327,24 @@ __global__ void __launch_bounds__(kLnThreads, 2) layernorm_i8_kernel(const int8_
     const uint32_t w[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
     const float4* g4 = reinterpret_cast<const float4*>(gamma + bj * 32 + c0);
     const float4* b4 = reinterpret_cast<const float4*>(beta + bj * 32 + c0);
-    float gm[16], bt[16];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 gg = __ldg(g4 + i), bb = __ldg(b4 + i);
-      gm[4 * i] = gg.x; gm[4 * i + 1] = gg.y; gm[4 * i + 2] = gg.z; gm[4 * i + 3] = gg.w;
-      bt[4 * i] = bb.x; bt[4 * i + 1] = bb.y; bt[4 * i + 2] = bb.z; bt[4 * i + 3] = bb.w;
-    }
     float v[32];
     float m = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float g[4];
-      i8x4_to_f32(w[i], g);
-      const float mu = i < 4 ? mean0 : mean1, rs = i < 4 ? rstd0 : rstd1;
+    for (int i = 0; i < 4; ++i) {  // columns 4i..4i+3 of the lane's 16, in both of its rows
+      const float4 gg = __ldg(g4 + i), bb = __ldg(b4 + i);
+      const float gm[4] = {gg.x, gg.y, gg.z, gg.w}, bt[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int c = (4 * i + j) & 15;
-        const float x = g[j] * sc;
-        const float y = fmaf((x - mu) * rs, gm[c], bt[c]);
-        v[4 * i + j] = y;
-        m = fmaxf(m, fabsf(y));
+      for (int k = 0; k < 2; ++k) {
+        float g[4];
+        i8x4_to_f32(w[i + 4 * k], g);
+        const float mu = k == 0 ? mean0 : mean1, rs = k == 0 ? rstd0 : rstd1;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float x = g[j] * sc;
+          const float y = fmaf((x - mu) * rs, gm[j], bt[j]);
+          v[4 * (i + 4 * k) + j] = y;
+          m = fmaxf(m, fabsf(y));
+        }
       }
     }
     const BlockQuant bq = block_quant(warp_max_nonneg(m));

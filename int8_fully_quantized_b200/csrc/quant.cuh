@@ -105,6 +105,16 @@ __device__ __forceinline__ void i8x4_to_f32(uint32_t w, float (&f)[4]) {
   for (int i = 0; i < 4; ++i) f[i] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7440 | i)) - 8388736.0f;
 }
 
+// Sum and sum of squares of the 16 signed INT8 codes of a 16-byte vector, exact (|sum| <= 2032,
+// sum of squares <= 258064), with 4-way byte dot products.
+__device__ __forceinline__ int chunk_sum_i8(const uint4& a) {
+  const int ones = 0x01010101;
+  return __dp4a(int(a.w), ones, __dp4a(int(a.z), ones, __dp4a(int(a.y), ones, __dp4a(int(a.x), ones, 0))));
+}
+__device__ __forceinline__ int chunk_sumsq_i8(const uint4& a) {
+  return __dp4a(int(a.w), int(a.w), __dp4a(int(a.z), int(a.z), __dp4a(int(a.y), int(a.y), __dp4a(int(a.x), int(a.x), 0))));
+}
+
 // Largest of 32 non-negative floats across the warp (non-negative floats order like their bits).
 __device__ __forceinline__ float warp_max_nonneg(float m) {
   return __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(m)));
