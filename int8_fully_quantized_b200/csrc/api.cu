@@ -167,7 +167,7 @@ int jf_quantize_block(const void* x, jf_dtype dt, int64_t rows, int64_t cols, in
     return JF_ERR_ALIAS;
   const DevInfo d = device_info();
   if (!d.ok) return JF_ERR_DEVICE;
-  return cuda_status(jf::launch_quantize(x, int(dt), rows, cols, q, s, d.sm_count, static_cast<cudaStream_t>(stream)));
+  return cuda_status(jf::launch_quantize(x, int(dt), rows, cols, q, s, d.status, d.sm_count, static_cast<cudaStream_t>(stream)));
 }
 
 int jf_dequantize_block(const int8_t* q, const float* s, int64_t rows, int64_t cols, void* y, jf_dtype dt,
@@ -345,7 +345,7 @@ int jf_quantize_granular(const void* x, jf_dtype dt, int64_t rows, int64_t cols,
   if (overlap(q, rows * cols, x, nx) || overlap(s, ns, x, nx) || overlap(q, rows * cols, s, ns)) return JF_ERR_ALIAS;
   const DevInfo d = device_info();
   if (!d.ok) return JF_ERR_DEVICE;
-  return cuda_status(jf::launch_quantize_granular(x, int(dt), rows, cols, int(g), q, s, d.sm_count,
+  return cuda_status(jf::launch_quantize_granular(x, int(dt), rows, cols, int(g), q, s, d.status, d.sm_count,
                                                   static_cast<cudaStream_t>(stream)));
 }
 

@@ -8,6 +8,7 @@
 // Layout: codes int8 [R, C] row-major, scales fp32 [R/32, C/32] row-major; block (I, J) covers
 // rows 32I..32I+31 and columns 32J..32J+31.
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -90,6 +91,135 @@ __global__ void __launch_bounds__(256, 3) quantize_kernel(const T* __restrict__ 
     }
     if (active && r0 == 0 && vc % HALF == 0) s[bi * nbc + bj] = bq.s;
   }
+}
+
+// ---------------------------------------------------------------------------------------------
+// a1, staged: the same quantizer with its input tiles brought in by TMA. One CTA of QtCfg::kWarps
+// warps per SM; each warp owns a ring of kDepth shared-memory slots and keeps that many of its 32 x 64
+// tiles in flight: its lane 0 issues a 2-D TMA tile load per tile, completion counted in bytes on
+// the slot's mbarrier. The warp waits for the oldest tile, copies its vectors to registers, refills
+// the slot with its tile kDepth ahead and quantizes from registers as above. The loads in flight no
+// longer depend on where the warps are in their arithmetic (measured at 65536 x 4096 bf16: 165 us
+// against 210 us with plain loads; 20 warps of two 4 KB slots beat 8, 16, 24 and 32 warps).
+// A tile whose second block lies past the last column (odd block-column count) is zero-filled there
+// by TMA and that half is not stored.
+// ---------------------------------------------------------------------------------------------
+template <typename T>
+struct QtCfg {  // 2-byte inputs: 4 KB tiles
+  static constexpr int kWarps = 20;
+  static constexpr int kDepth = 2;
+};
+template <>
+struct QtCfg<float> {  // 8 KB tiles
+  static constexpr int kWarps = 12;
+  static constexpr int kDepth = 2;
+};
+template <typename T>
+__host__ __device__ constexpr int qt_tile_bytes() { return 32 * 64 * int(sizeof(T)); }
+template <typename T>
+__host__ __device__ constexpr int qt_smem_bytes() { return QtCfg<T>::kWarps * QtCfg<T>::kDepth * qt_tile_bytes<T>() + 128; }
+
+template <typename T>
+__global__ void __launch_bounds__(32 * QtCfg<T>::kWarps, 1) quantize_tma_kernel(const __grid_constant__ CUtensorMap map,
+                                                                              int64_t R, int64_t C, int8_t* __restrict__ q,
+                                                                              float* __restrict__ s, unsigned int* status) {
+  constexpr int EPV = Vec<T>::kElems;
+  constexpr int VPR = 64 / EPV;
+  constexpr int RSTEP = 32 / VPR;
+  constexpr int HALF = VPR / 2;
+  constexpr int VPG = 8 / EPV;
+  constexpr int ROW = 64 * int(sizeof(T));  // bytes of one tile row in shared memory
+  constexpr int TILE = qt_tile_bytes<T>();
+  constexpr int DEPTH = QtCfg<T>::kDepth;
+  constexpr int kQtWarps = QtCfg<T>::kWarps;
+  constexpr int kQtRingBytes = DEPTH * TILE;
+  static_assert(qt_smem_bytes<T>() <= 227 * 1024, "the rings fit one SM's shared memory");
+  extern __shared__ uint8_t qt_smem_raw[];
+  __shared__ uint64_t bars[kQtWarps][DEPTH];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // TMA tile destinations: 128-byte aligned (the launch asks for 128 spare bytes)
+  uint8_t* qt_smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(qt_smem_raw) + 127) & ~uintptr_t(127));
+  uint8_t* ring = qt_smem + warp * kQtRingBytes;
+  uint64_t* bar = bars[warp];
+  const int64_t nbc = C >> 5;
+  const int64_t npc = (nbc + 1) >> 1;
+  const int64_t npairs = (R >> 5) * npc;
+  const int64_t gw = int64_t(blockIdx.x) * kQtWarps + warp, nw = int64_t(gridDim.x) * kQtWarps;
+  const int64_t n_my = gw < npairs ? (npairs - gw + nw - 1) / nw : 0;  // this warp's tiles gw, gw + nw, ...
+  if (lane == 0) {
+    for (int d = 0; d < DEPTH; ++d) mbar_init(&bar[d], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  auto issue = [&](int64_t i) {  // lane 0: the warp's i-th tile into slot i % DEPTH
+    const int64_t p = gw + i * nw;
+    const int64_t bi = p / npc, pj = p - bi * npc;
+    uint64_t* b = &bar[i % DEPTH];
+    mbar_arrive_expect_tx(b, TILE);
+    tma_load_2d(ring + (i % DEPTH) * TILE, &map, b, int(pj * 64), int(bi * 32));
+  };
+  if (lane == 0)
+    for (int64_t i = 0; i < n_my && i < DEPTH; ++i) issue(i);
+  const int r0 = lane / VPR, vc = lane % VPR;
+  const int half = vc / HALF;
+  uint32_t no_abort = 0u;
+  int64_t i = 0;
+  for (; i < n_my; ++i) {
+    const int slot = int(i % DEPTH);
+    const uint32_t ph = uint32_t(i / DEPTH) & 1u;
+    const bool ok = mbar_try_wait(&bar[slot], ph) || mbar_wait(&bar[slot], ph, &no_abort, status);
+    if (!__all_sync(0xffffffffu, ok)) break;
+    const uint8_t* tile = ring + slot * TILE;
+    uint4 raw[VPR];
+#pragma unroll
+    for (int t = 0; t < VPR; ++t) raw[t] = *reinterpret_cast<const uint4*>(tile + (r0 + t * RSTEP) * ROW + vc * 16);
+    __syncwarp();  // every lane has its vectors: the slot may be refilled
+    if (lane == 0 && i + DEPTH < n_my) {
+      fence_proxy_async_smem();  // the lanes' reads of the slot precede the TMA write into it
+      issue(i + DEPTH);
+    }
+    const int64_t p = gw + i * nw;
+    const int64_t bi = p / npc, pj = p - bi * npc;
+    const int64_t bj = 2 * pj + half;
+    const bool active = bj < nbc;
+    uint32_t mb = 0;
+#pragma unroll
+    for (int t = 0; t < VPR; ++t) {
+      const uint32_t w[4] = {raw[t].x, raw[t].y, raw[t].z, raw[t].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if constexpr (EPV == 4) mb = max(mb, w[k] & 0x7FFFFFFFu);
+        else mb = __vmaxu2(mb, w[k] & 0x7FFF7FFFu);
+      }
+    }
+    if constexpr (EPV != 4) mb = max(mb & 0xFFFFu, mb >> 16);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1)
+      if (o != HALF) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+    const BlockQuant bq = block_quant(abs_max_of_bits<T>(mb));
+    int8_t* dst = q + (bi * 32 + r0) * C + pj * 64 + vc * EPV;
+#pragma unroll
+    for (int t = 0; t < VPR; t += VPG) {
+      float v[8];
+#pragma unroll
+      for (int g = 0; g < VPG; ++g) Vec<T>::unpack(raw[t + g], *reinterpret_cast<float(*)[EPV]>(v + g * EPV));
+      uint32_t w[2];
+      quant_pack<8>(v, bq, w);
+      if (active) {
+        if constexpr (EPV == 4) {
+          *reinterpret_cast<uint32_t*>(dst + int64_t(t) * RSTEP * C) = w[0];
+          *reinterpret_cast<uint32_t*>(dst + int64_t(t + 1) * RSTEP * C) = w[1];
+        } else {
+          *reinterpret_cast<uint2*>(dst + int64_t(t) * RSTEP * C) = make_uint2(w[0], w[1]);
+        }
+      }
+    }
+    if (active && r0 == 0 && vc % HALF == 0) s[bi * nbc + bj] = bq.s;
+  }
+  // after a wait that ran out, the tiles still in flight land before the CTA exits
+  if (lane == 0)
+    for (int64_t j = i; j < n_my && j < i + DEPTH; ++j) mbar_wait_teardown(&bar[j % DEPTH], uint32_t(j / DEPTH) & 1u, status);
+  __syncwarp();
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -368,8 +498,52 @@ static int grid_for_blocks(int64_t nblocks, int sm_count) {
   return int(ctas < 1 ? 1 : ctas);
 }
 
-cudaError_t launch_quantize(const void* x, int dtype, int64_t R, int64_t C, int8_t* q, float* s, int sm_count,
-                            cudaStream_t st) {
+// 2-D tensor map over the row-major [R, C] input with 32-row x 64-column boxes, no swizzle.
+static bool make_quant_map(CUtensorMap* m, const void* x, int dtype, int64_t R, int64_t C) {
+  auto fn = tensor_map_encoder();
+  if (fn == nullptr) return false;
+  const CUtensorMapDataType dt = dtype == 0 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : dtype == 1 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const uint64_t esz = dtype == 0 ? 4 : 2;
+  cuuint64_t dims[2] = {cuuint64_t(C), cuuint64_t(R)};
+  cuuint64_t strides[1] = {cuuint64_t(C) * esz};
+  cuuint32_t box[2] = {64, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+template <typename T>
+static cudaError_t run_quantize_tma(const CUtensorMap& map, int64_t R, int64_t C, int8_t* q, float* s,
+                                    unsigned int* status, int sm_count, cudaStream_t st) {
+  static unsigned long long attr_set = 0;  // one bit per device ordinal
+  auto kern = quantize_tma_kernel<T>;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attr_set & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, qt_smem_bytes<T>());
+    if (e != cudaSuccess) return e;
+    attr_set |= bit;
+  }
+  const int64_t npairs = (R / 32) * ((C / 32 + 1) / 2);
+  int64_t grid = (npairs + QtCfg<T>::kWarps - 1) / QtCfg<T>::kWarps;
+  if (grid > sm_count) grid = sm_count;
+  kern<<<int(grid), 32 * QtCfg<T>::kWarps, qt_smem_bytes<T>(), st>>>(map, R, C, q, s, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(const void* x, int dtype, int64_t R, int64_t C, int8_t* q, float* s,
+                            unsigned int* status, int sm_count, cudaStream_t st) {
+  CUtensorMap map;
+  if (status != nullptr && make_quant_map(&map, x, dtype, R, C)) {
+    if (dtype == 0) return run_quantize_tma<float>(map, R, C, q, s, status, sm_count, st);
+    if (dtype == 1) return run_quantize_tma<__nv_bfloat16>(map, R, C, q, s, status, sm_count, st);
+    return run_quantize_tma<__half>(map, R, C, q, s, status, sm_count, st);
+  }
+  // no tensor map for this input (the driver refused it): plain loads
   const int grid = grid_for_blocks((R / 32) * ((C / 32 + 1) / 2), sm_count);  // one warp per block pair
   if (dtype == 0)
     quantize_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), R, C, q, s);

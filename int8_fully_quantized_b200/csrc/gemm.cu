@@ -334,7 +334,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_co
 // ---------------------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------------------
-static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (fn == nullptr) {
     void* ptr = nullptr;
@@ -349,7 +349,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 2-D int8 tensor map over a row-major [outer, inner] matrix with row pitch `ld` bytes.
 static bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
                      uint32_t box_inner, uint32_t box_outer) {
-  auto fn = encode_fn();
+  auto fn = tensor_map_encoder();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {ld};

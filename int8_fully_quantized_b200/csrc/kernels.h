@@ -2,12 +2,17 @@
 #pragma once
 #include <cstdint>
 #include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 namespace jf {
 
-cudaError_t launch_quantize(const void* x, int dtype, int64_t R, int64_t C, int8_t* q, float* s, int sm_count,
-                            cudaStream_t st);
+// The driver's cuTensorMapEncodeTiled (null if the driver does not provide it).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
+// `status`: the device status word, raised when a bounded wait in the kernel runs out.
+cudaError_t launch_quantize(const void* x, int dtype, int64_t R, int64_t C, int8_t* q, float* s,
+                            unsigned int* status, int sm_count, cudaStream_t st);
 cudaError_t launch_dequantize(const int8_t* q, const float* s, int64_t R, int64_t C, void* y, int dtype,
                               int sm_count, cudaStream_t st);
 cudaError_t launch_gelu_i8(const int8_t* q, const float* s, int64_t R, int64_t C, int8_t* qo, float* so,
@@ -27,7 +32,7 @@ cudaError_t launch_mx_gemm(const uint8_t* a_q, const uint8_t* a_s, const uint8_t
 // block [R/32, C/32], token [R], channel [C], tensor [1].
 enum Granularity { kGranBlock = 0, kGranToken = 1, kGranChannel = 2, kGranTensor = 3 };
 cudaError_t launch_quantize_granular(const void* x, int dtype, int64_t R, int64_t C, int g, int8_t* q, float* s,
-                                     int sm_count, cudaStream_t st);
+                                     unsigned int* status, int sm_count, cudaStream_t st);
 cudaError_t launch_dequantize_granular(const int8_t* q, const float* s, int64_t R, int64_t C, int g, void* y,
                                        int dtype, int sm_count, cudaStream_t st);
 cudaError_t launch_quant_error(const void* x, int dtype, const int8_t* q, const float* s, int64_t R, int64_t C, int g,

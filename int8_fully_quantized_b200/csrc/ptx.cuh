@@ -77,6 +77,9 @@ __device__ __forceinline__ void mbar_wait_teardown(uint64_t* bar, uint32_t parit
 }
 
 // ---------------------------------------------------------------- async copies
+// Orders this thread's (and, after a warp or CTA barrier, its peers') generic-proxy accesses to
+// shared memory before its subsequent async-proxy (TMA) accesses to it.
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 // 2-D TMA tile load into shared memory, completion counted in bytes on `bar`.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
   asm volatile(
