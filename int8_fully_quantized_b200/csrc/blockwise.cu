@@ -385,9 +385,9 @@ __global__ void __launch_bounds__(32 * kGeluWarps, 3) gelu_i8_kernel(const int8_
 //            integer sums of each 16-code chunk (one block scale per chunk) scaled and accumulated
 //            in fp64, then mean, biased variance and rstd = 1 / sqrt(var + eps) in fp64, kept in
 //            shared memory.
-//   phase 2: warp w handles column blocks w, w + 16, ...: y = (x - mean) * rstd * gamma + beta in
-//            fp32, block absmax, per-block re-quantization. The strip is read a second time; it
-//            is at most 32 * H bytes and is still in L2.
+//   phase 2: warp w handles column blocks w, w + 16, ...: y = (q (s rstd) - mean rstd) gamma + beta
+//            in fp32 (two FMAs per element), block absmax, per-block re-quantization. The strip is
+//            read a second time; it is at most 32 * H bytes and is still in L2.
 // ---------------------------------------------------------------------------------------------
 constexpr int kLnThreads = 512;
 
@@ -457,6 +457,8 @@ __global__ void __launch_bounds__(kLnThreads, 2) layernorm_i8_kernel(const int8_
     const uint32_t w[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
     const float4* g4 = reinterpret_cast<const float4*>(gamma + bj * 32 + c0);
     const float4* b4 = reinterpret_cast<const float4*>(beta + bj * 32 + c0);
+    // xhat = (q s - mean) rstd = q (s rstd) - mean rstd: one FMA per element
+    const float a0f = sc * rstd0, b0f = -mean0 * rstd0, a1f = sc * rstd1, b1f = -mean1 * rstd1;
     float v[32];
     float m = 0.0f;
 #pragma unroll
@@ -467,11 +469,10 @@ __global__ void __launch_bounds__(kLnThreads, 2) layernorm_i8_kernel(const int8_
       for (int k = 0; k < 2; ++k) {
         float g[4];
         i8x4_to_f32(w[i + 4 * k], g);
-        const float mu = k == 0 ? mean0 : mean1, rs = k == 0 ? rstd0 : rstd1;
+        const float af = k == 0 ? a0f : a1f, bf = k == 0 ? b0f : b1f;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float x = g[j] * sc;
-          const float y = fmaf((x - mu) * rs, gm[j], bt[j]);
+          const float y = fmaf(fmaf(g[j], af, bf), gm[j], bt[j]);
           v[4 * (i + 4 * k) + j] = y;
           m = fmaxf(m, fabsf(y));
         }
