@@ -192,7 +192,7 @@ JF_API int jf_layernorm_i8_bwd(jf_cqtensor X, jf_cqtensor dY, const float* gamma
                                void* stream);
 
 /* Bytes of workspace jf_layernorm_i8_bwd needs for X of [rows, cols]:
- * min(rows / 32, 444) * 2 * cols * 4, or -1 for an invalid shape (cols > 24576 included). */
+ * min(rows / 32, 296) * 2 * cols * 4, or -1 for an invalid shape (cols > 24576 included). */
 JF_API int64_t jf_layernorm_i8_bwd_workspace_bytes(int64_t rows, int64_t cols);
 
 /*

@@ -78,7 +78,8 @@ __global__ void __launch_bounds__(32 * kGeluBwdWarps, 3) gelu_i8_bwd_kernel(
 // LayerNorm_i8 backward. For the layer y = (x - mu) rstd gamma + beta (mu, biased variance over the
 // H columns of a row, rstd = 1 / sqrt(var + eps)), with xhat = (x - mu) rstd and g = dy gamma:
 //   dx = rstd (g - mean(g) - xhat mean(g xhat)),  dgamma = sum_rows dy xhat,  dbeta = sum_rows dy.
-// Persistent CTAs of 8 warps, three per SM, each looping over 32-row strips:
+// Persistent CTAs of 8 warps, two per SM (three spill registers and ran 5% slower), each looping over
+// 32-row strips:
 //   phase 1: warp w reduces rows w, w + 8, w + 16 and w + 24 of the strip, each in one pass: sums
 //            of x, x^2, g and g x over 16-value chunks (the x sums exact in integers, the g sums in
 //            fp32 before the block scales), scaled and accumulated in fp64. Then mean, rstd, mean(g) and
@@ -90,13 +91,13 @@ __global__ void __launch_bounds__(32 * kGeluBwdWarps, 3) gelu_i8_bwd_kernel(
 //   When gamma or beta gradients are asked for, a CTA adds each strip's column sums into fp32
 //   accumulators in shared memory (every column belongs to one warp, so no atomics), writes them
 //   to part[cta][0 | 1][H] at the end, and ln_bwd_reduce_kernel adds the CTAs' partials in a fixed
-//   order. The workspace is ln_bwd_ctas(R) * 2 * H floats, independent of R beyond 444 strips.
+//   order. The workspace is ln_bwd_ctas(R) * 2 * H floats, independent of R beyond 296 strips.
 // ---------------------------------------------------------------------------------------------
 constexpr int kLnbThreads = 256;
 
 int64_t ln_bwd_ctas(int64_t R) { return R / 32 < kLnBwdMaxCtas ? R / 32 : kLnBwdMaxCtas; }
 
-__global__ void __launch_bounds__(kLnbThreads, 3) layernorm_i8_bwd_kernel(
+__global__ void __launch_bounds__(kLnbThreads, 2) layernorm_i8_bwd_kernel(
     const int8_t* __restrict__ xq, const float* __restrict__ xs, const int8_t* __restrict__ dq,
     const float* __restrict__ ds, int64_t R, int64_t H, const float* __restrict__ gamma, float eps,
     int8_t* __restrict__ qo, float* __restrict__ so, float* __restrict__ part) {
@@ -204,9 +205,10 @@ __global__ void __launch_bounds__(kLnbThreads, 3) layernorm_i8_bwd_kernel(
         i8x4_to_f32(wx[i], fx);
         i8x4_to_f32(wd[i], fd);
         const float4 st = s_stat[rg + 4 * i];
+        const float ax = sx * st.y, bx = -st.x * st.y;  // xhat = q (s rstd) - mean rstd
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float xhat = (fx[j] * sx - st.x) * st.y;
+          const float xhat = fmaf(fx[j], ax, bx);
           const float dy = fd[j] * sd;
           const float dx = st.y * (fmaf(dy, gm[j], -st.z) - xhat * st.w);
           v[4 * i + j] = dx;

@@ -40,7 +40,7 @@ cudaError_t launch_quant_error(const void* x, int dtype, const int8_t* q, const 
 
 // INT8 backward of GELU_i8 and LayerNorm_i8 (backward.cu). `part` is the fp32 workspace of
 // per-CTA column sums, [ln_bwd_ctas(R)][2][H]; null when neither dgamma nor dbeta is wanted.
-constexpr int64_t kLnBwdMaxCtas = 444;   // three resident CTAs on each of 148 SMs
+constexpr int64_t kLnBwdMaxCtas = 296;   // two resident CTAs on each of 148 SMs
 constexpr int64_t kLnBwdMaxCols = 24576; // the [2][H] fp32 accumulators fit in one SM's shared memory
 int64_t ln_bwd_ctas(int64_t R);
 // Size of the static scratch the allocation-free LayerNorm backward uses in place of a workspace,
