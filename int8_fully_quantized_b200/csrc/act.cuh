@@ -38,4 +38,15 @@ __device__ __forceinline__ float gelu_grad_f32(float x) {
   return fmaf(x * 0.39894228040143267794f, expf(-0.5f * x * x), Phi);
 }
 
+// GELU'(x) and GELU'(-x) for x >= 0 from one erfc and one exp: Phi(-x) = 1 - Phi(x) and phi is even,
+// so both share e = erfc(x / sqrt 2) and exp(-x^2 / 2). Each result is bit-identical to
+// gelu_grad_f32 of the same argument (the sign flips involved are exact).
+__device__ __forceinline__ void gelu_grad_pair_f32(float x, float& at_pos, float& at_neg) {
+  const float e = erfc_nonneg(x * 0.70710678118654752440f);
+  const float ex = expf(-0.5f * x * x);
+  const float xc = x * 0.39894228040143267794f;
+  at_pos = fmaf(xc, ex, 0.5f * (2.0f - e));
+  at_neg = fmaf(-xc, ex, 0.5f * e);
+}
+
 }  // namespace jf

@@ -19,8 +19,9 @@ namespace jf {
 // ---------------------------------------------------------------------------------------------
 // GELU_i8 backward: dx = fp32(dy) * GELU'(fp32(x)) per element, re-quantized per block. One warp
 // per block, lane l takes columns 16 (l % 2) .. +15 of rows l / 2 and 16 + l / 2 (two 16-byte
-// chunks per tensor). A block of x has at most 255 distinct values q * s, so the warp tabulates
-// GELU' of all of them first (8 evaluations per lane instead of 32) and looks its values up.
+// chunks per tensor). A block of x has at most 256 distinct values q * s, so the warp tabulates
+// GELU' of all of them first (4 erfc/exp evaluations per lane, each serving a code and its
+// negation, instead of 32) and looks its values up.
 // ---------------------------------------------------------------------------------------------
 constexpr int kGeluBwdWarps = 8;
 
@@ -42,12 +43,16 @@ __global__ void __launch_bounds__(32 * kGeluBwdWarps, 3) gelu_i8_bwd_kernel(
     const uint4 a1 = ld_stream_v4(xq + off + 16 * C);
     const uint4 d0 = ld_stream_v4(dq + off);
     const uint4 d1 = ld_stream_v4(dq + off + 16 * C);
-    // table[u] = GELU'(fp32(u - 128) * sx) for the code u - 128
+    // table[u] = GELU'(fp32(u - 128) * sx) for the code u - 128; one evaluation serves m and -m
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int u = lane + 32 * j;
-      tab[u] = gelu_grad_f32(float(u - 128) * sx);
+    for (int j = 0; j < 4; ++j) {
+      const int m = lane + 32 * j;  // |code| 0..127
+      float gp, gn;
+      gelu_grad_pair_f32(float(m) * sx, gp, gn);
+      tab[128 + m] = gp;
+      if (m != 0) tab[128 - m] = gn;
     }
+    if (lane == 0) tab[0] = gelu_grad_f32(-128.0f * sx);  // code -128
     __syncwarp();
     const uint32_t wx[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
     const uint32_t wd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
