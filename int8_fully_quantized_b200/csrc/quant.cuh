@@ -58,9 +58,30 @@ __device__ __forceinline__ uint32_t quant_byte(float x, const BlockQuant& b) {
   return quant_byte_exact(x, b.s);
 }
 
+// The fast path of quant_byte for two values at once, in packed fp32x2 arithmetic (sm_100): per
+// value t = RN(x * inv), tp = RN(t + kRoundMagic) (its low byte is the code) and d = t - round(t),
+// each operation rounded exactly as its scalar form, so the results are bit-identical. Packing
+// halves the issue slots of these four operations.
+__device__ __forceinline__ void round_pair_fast(float x0, float x1, float inv, float& tp0, float& tp1, float& d0,
+                                                float& d1) {
+  asm("{\n\t.reg .b64 x, iv, m, t, tp, r, d;\n\t"
+      "mov.b64 x, {%4, %5};\n\t"
+      "mov.b64 iv, {%6, %6};\n\t"
+      "mov.b64 m, {%7, %7};\n\t"
+      "mul.rn.f32x2 t, x, iv;\n\t"
+      "add.rn.f32x2 tp, t, m;\n\t"
+      "sub.rn.f32x2 r, tp, m;\n\t"
+      "sub.rn.f32x2 d, t, r;\n\t"
+      "mov.b64 {%0, %1}, tp;\n\t"
+      "mov.b64 {%2, %3}, d;\n\t}"
+      : "=f"(tp0), "=f"(tp1), "=f"(d0), "=f"(d1)
+      : "f"(x0), "f"(x1), "f"(inv), "f"(kRoundMagic));
+}
+
 // Codes of N values (N a multiple of 8), packed four to a word (value 4i in byte 0 of word i).
-// The fast path of quant_byte runs branch-free on groups of 8 values; one test per group looks for a
-// value next to a rounding tie (rare), and only then is the group recomputed exactly.
+// The fast path of quant_byte runs branch-free on groups of 8 values (in packed pairs); one test per
+// group looks for a value next to a rounding tie (rare), and only then is the group recomputed
+// exactly.
 template <int N>
 __device__ __forceinline__ void quant_pack(const float* v, const BlockQuant& b, uint32_t* out) {
   static_assert(N % 8 == 0, "values are handled in groups of eight");
@@ -70,11 +91,12 @@ __device__ __forceinline__ void quant_pack(const float* v, const BlockQuant& b, 
     if (b.mode == 2) {
       bool near_tie = false;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float t = v[g + i] * b.inv;
-        const float tp = t + kRoundMagic;
-        near_tie |= !(fabsf(t - (tp - kRoundMagic)) < 0.49993896484375f);  // 0.5 - 2^-14
-        c[i] = __float_as_uint(tp);
+      for (int i = 0; i < 8; i += 2) {
+        float tp0, tp1, d0, d1;
+        round_pair_fast(v[g + i], v[g + i + 1], b.inv, tp0, tp1, d0, d1);
+        near_tie |= !(fabsf(d0) < 0.49993896484375f) | !(fabsf(d1) < 0.49993896484375f);  // 0.5 - 2^-14
+        c[i] = __float_as_uint(tp0);
+        c[i + 1] = __float_as_uint(tp1);
       }
       if (near_tie) {
 #pragma unroll
