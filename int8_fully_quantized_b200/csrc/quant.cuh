@@ -120,11 +120,23 @@ __device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, ui
 }
 
 // Four signed INT8 codes (bytes of w) -> four exact fp32 values. Flipping the sign bit gives
-// q + 128 as an unsigned byte u; the fp32 with bit pattern 0x4B0000uu is 2^23 + u exactly.
+// q + 128 as an unsigned byte u; the fp32 with bit pattern 0x4B0000uu is 2^23 + u exactly, and one
+// exact subtraction of 2^23 + 128 (two values per packed fp32x2 instruction) leaves q.
 __device__ __forceinline__ void i8x4_to_f32(uint32_t w, float (&f)[4]) {
   const uint32_t u = w ^ 0x80808080u;
+  uint32_t b[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) f[i] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7440 | i)) - 8388736.0f;
+  for (int i = 0; i < 4; ++i) b[i] = __byte_perm(u, 0x4B000000u, 0x7440 | i);
+  asm("{\n\t.reg .b64 lo, hi, m;\n\t"
+      "mov.b64 lo, {%4, %5};\n\t"
+      "mov.b64 hi, {%6, %7};\n\t"
+      "mov.b64 m, {%8, %8};\n\t"
+      "sub.rn.f32x2 lo, lo, m;\n\t"
+      "sub.rn.f32x2 hi, hi, m;\n\t"
+      "mov.b64 {%0, %1}, lo;\n\t"
+      "mov.b64 {%2, %3}, hi;\n\t}"
+      : "=f"(f[0]), "=f"(f[1]), "=f"(f[2]), "=f"(f[3])
+      : "r"(b[0]), "r"(b[1]), "r"(b[2]), "r"(b[3]), "f"(8388736.0f));
 }
 
 // Sum and sum of squares of the 16 signed INT8 codes of a 16-byte vector, exact (|sum| <= 2032,
