@@ -64,9 +64,11 @@ __global__ void __launch_bounds__(32 * kGeluBwdWarps, 3) gelu_i8_bwd_kernel(
       float g[4];
       i8x4_to_f32(wd[i], g);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        v[4 * i + j] = (g[j] * sd) * tab[(u >> (8 * j)) & 0xFFu];
-        m = fmaxf(m, fabsf(v[4 * i + j]));
+      for (int j = 0; j < 4; j += 2) {  // (g sd) GELU'(x), two values per packed instruction
+        float d0, d1;
+        mul_x2(g[j], g[j + 1], sd, sd, d0, d1);
+        mul_x2(d0, d1, tab[(u >> (8 * j)) & 0xFFu], tab[(u >> (8 * j + 8)) & 0xFFu], v[4 * i + j], v[4 * i + j + 1]);
+        m = fmaxf(m, fmaxf(fabsf(v[4 * i + j]), fabsf(v[4 * i + j + 1])));
       }
     }
     __syncwarp();  // the table is rewritten for the next block only after every lane has read it
@@ -148,7 +150,7 @@ __global__ void __launch_bounds__(kLnbThreads, 2) layernorm_i8_bwd_kernel(
           const uint32_t wd[4] = {dv[u].x, dv[u].y, dv[u].z, dv[u].w};
           const float4* g4 = reinterpret_cast<const float4*>(gamma + ch * 16);
           // the chunk's codes share one block scale per tensor: the scales are applied once per chunk
-          float pg = 0.0f, pgx = 0.0f;  // sums of q_dy gamma and q_dy gamma q_x over the chunk
+          float pg2[2] = {0.0f, 0.0f}, pgx2[2] = {0.0f, 0.0f};  // sums of q_dy gamma and q_dy gamma q_x
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const float4 gm = __ldg(g4 + i);
@@ -156,18 +158,20 @@ __global__ void __launch_bounds__(kLnbThreads, 2) layernorm_i8_bwd_kernel(
             float fx[4], fd[4];
             i8x4_to_f32(wx[i], fx);
             i8x4_to_f32(wd[i], fd);
+            // per column pair: t = q_dy gamma, pg += t, pgx += t q_x (packed pairs, two partial sums each)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float t = fd[j] * gmv[j];
-              pg += t;
-              pgx = fmaf(t, fx[j], pgx);
+            for (int j = 0; j < 4; j += 2) {
+              float t0, t1;
+              mul_x2(fd[j], fd[j + 1], gmv[j], gmv[j + 1], t0, t1);
+              add_x2(pg2[0], pg2[1], t0, t1, pg2[0], pg2[1]);
+              fma_x2(t0, t1, fx[j], fx[j + 1], pgx2[0], pgx2[1], pgx2[0], pgx2[1]);
             }
           }
           const double sx = double(scx[u]), sd = double(scd[u]);
           sum_x = fma(sx, double(chunk_sum_i8(av[u])), sum_x);  // exact integer sums of the x codes
           sum_xx = fma(sx * sx, double(chunk_sumsq_i8(av[u])), sum_xx);
-          sum_g = fma(sd, double(pg), sum_g);
-          sum_gx = fma(sd * sx, double(pgx), sum_gx);
+          sum_g = fma(sd, double(pg2[0] + pg2[1]), sum_g);
+          sum_gx = fma(sd * sx, double(pgx2[0] + pgx2[1]), sum_gx);
         }
       }
 #pragma unroll
@@ -211,15 +215,18 @@ __global__ void __launch_bounds__(kLnbThreads, 2) layernorm_i8_bwd_kernel(
         i8x4_to_f32(wd[i], fd);
         const float4 st = s_stat[rg + 4 * i];
         const float ax = sx * st.y, bx = -st.x * st.y;  // xhat = q (s rstd) - mean rstd
+        // dx = rstd (dy gamma - mean(g) - xhat mean(g xhat)), in packed pairs of columns
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float xhat = fmaf(fx[j], ax, bx);
-          const float dy = fd[j] * sd;
-          const float dx = st.y * (fmaf(dy, gm[j], -st.z) - xhat * st.w);
-          v[4 * i + j] = dx;
-          m = fmaxf(m, fabsf(dx));
-          pgam[j] = fmaf(dy, xhat, pgam[j]);
-          pbet[j] += dy;
+        for (int j = 0; j < 4; j += 2) {
+          float xh0, xh1, dy0, dy1, t0, t1, u0, u1;
+          fma_x2(fx[j], fx[j + 1], ax, ax, bx, bx, xh0, xh1);
+          mul_x2(fd[j], fd[j + 1], sd, sd, dy0, dy1);
+          fma_x2(dy0, dy1, gm[j], gm[j + 1], -st.z, -st.z, t0, t1);
+          fma_x2(xh0, xh1, -st.w, -st.w, t0, t1, u0, u1);
+          mul_x2(u0, u1, st.y, st.y, v[4 * i + j], v[4 * i + j + 1]);
+          m = fmaxf(m, fmaxf(fabsf(v[4 * i + j]), fabsf(v[4 * i + j + 1])));
+          fma_x2(dy0, dy1, xh0, xh1, pgam[j], pgam[j + 1], pgam[j], pgam[j + 1]);
+          add_x2(pbet[j], pbet[j + 1], dy0, dy1, pbet[j], pbet[j + 1]);
         }
       }
       const BlockQuant bq = block_quant(warp_max_nonneg(m));

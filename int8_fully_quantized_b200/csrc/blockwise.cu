@@ -260,8 +260,8 @@ __global__ void __launch_bounds__(256, 4) dequantize_kernel(const int8_t* __rest
       for (int i = 0; i < EPV / 4; ++i) {
         float g[4];
         i8x4_to_f32(w[t][i], g);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) f[4 * i + j] = g[j] * sc;
+        mul_x2(g[0], g[1], sc, sc, f[4 * i], f[4 * i + 1]);
+        mul_x2(g[2], g[3], sc, sc, f[4 * i + 2], f[4 * i + 3]);
       }
       *reinterpret_cast<uint4*>(dst + int64_t(t) * RSTEP * C) = Vec<T>::pack(f);
     }
@@ -471,10 +471,12 @@ __global__ void __launch_bounds__(kLnThreads, 2) layernorm_i8_kernel(const int8_
         i8x4_to_f32(w[i + 4 * k], g);
         const float af = k == 0 ? a0f : a1f, bf = k == 0 ? b0f : b1f;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float y = fmaf(fmaf(g[j], af, bf), gm[j], bt[j]);
-          v[4 * (i + 4 * k) + j] = y;
-          m = fmaxf(m, fabsf(y));
+        for (int j = 0; j < 4; j += 2) {  // two columns per packed instruction
+          float xh0, xh1;
+          float* y = v + 4 * (i + 4 * k) + j;
+          fma_x2(g[j], g[j + 1], af, af, bf, bf, xh0, xh1);
+          fma_x2(xh0, xh1, gm[j], gm[j + 1], bt[j], bt[j + 1], y[0], y[1]);
+          m = fmaxf(m, fmaxf(fabsf(y[0]), fabsf(y[1])));
         }
       }
     }

@@ -119,6 +119,27 @@ __device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, ui
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
+// Packed fp32x2 elementwise arithmetic (sm_100): (d0, d1) = (a0 op b0 [+ c0], a1 op b1 [+ c1]), each
+// lane rounded to nearest exactly as the scalar instruction, in half the issue slots.
+__device__ __forceinline__ void fma_x2(float a0, float a1, float b0, float b1, float c0, float c1, float& d0, float& d1) {
+  asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void mul_x2(float a0, float a1, float b0, float b1, float& d0, float& d1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void add_x2(float a0, float a1, float b0, float b1, float& d0, float& d1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // Four signed INT8 codes (bytes of w) -> four exact fp32 values. Flipping the sign bit gives
 // q + 128 as an unsigned byte u; the fp32 with bit pattern 0x4B0000uu is 2^23 + u exactly, and one
 // exact subtraction of 2^23 + 128 (two values per packed fp32x2 instruction) leaves q.
