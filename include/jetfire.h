@@ -93,7 +93,9 @@ typedef enum { JF_GRAN_BLOCK = 0, JF_GRAN_TOKEN = 1, JF_GRAN_CHANNEL = 2, JF_GRA
  *   s     device, fp32 [rows/32, cols/32], 4-byte aligned (output)
  * Codes and scales are bit-exact with the rule above (bf16/fp16 are widened exactly first).
  * The kernel stages x through shared memory with TMA tile loads and waits on them with bounded
- * waits: if one runs out, the kernel gives up and jf_device_status reports JF_ERR_TIMEOUT.
+ * waits: if one runs out, the kernel gives up and jf_device_status reports JF_ERR_TIMEOUT. With
+ * JF_PLAIN_LOADS=1 in the environment (read on every call) a kernel with plain loads runs instead
+ * (the path for inputs the driver cannot describe with a tensor map); its results are identical.
  */
 JF_API int jf_quantize_block(const void* x, jf_dtype dt, int64_t rows, int64_t cols, int8_t* q, float* s,
                       void* stream);

@@ -1,5 +1,6 @@
 // C ABI of the library: argument validation, then the kernel launch (see include/jetfire.h).
 #include <cstdint>
+#include <cstdlib>
 #include <cuda_runtime.h>
 
 #include "jetfire.h"
@@ -61,6 +62,13 @@ inline bool overlap(const void* a, int64_t na, const void* b, int64_t nb) {
 }
 inline int64_t elem_size(jf_dtype dt) { return dt == JF_F32 ? 4 : 2; }
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? JF_OK : JF_ERR_CUDA; }
+
+// JF_PLAIN_LOADS=1 in the environment (read on every call) selects the quantizer's plain-load kernel,
+// which otherwise serves only inputs the driver will not describe with a TMA tensor map.
+inline bool plain_loads_forced() {
+  const char* v = std::getenv("JF_PLAIN_LOADS");
+  return v != nullptr && v[0] == '1';
+}
 
 int check_cq(const jf_cqtensor& t) {
   if (!dims_ok(t.rows, t.cols)) return JF_ERR_SHAPE;
@@ -167,7 +175,8 @@ int jf_quantize_block(const void* x, jf_dtype dt, int64_t rows, int64_t cols, in
     return JF_ERR_ALIAS;
   const DevInfo d = device_info();
   if (!d.ok) return JF_ERR_DEVICE;
-  return cuda_status(jf::launch_quantize(x, int(dt), rows, cols, q, s, d.status, d.sm_count, static_cast<cudaStream_t>(stream)));
+  return cuda_status(jf::launch_quantize(x, int(dt), rows, cols, q, s, plain_loads_forced() ? nullptr : d.status,
+                                          d.sm_count, static_cast<cudaStream_t>(stream)));
 }
 
 int jf_dequantize_block(const int8_t* q, const float* s, int64_t rows, int64_t cols, void* y, jf_dtype dt,
@@ -345,7 +354,8 @@ int jf_quantize_granular(const void* x, jf_dtype dt, int64_t rows, int64_t cols,
   if (overlap(q, rows * cols, x, nx) || overlap(s, ns, x, nx) || overlap(q, rows * cols, s, ns)) return JF_ERR_ALIAS;
   const DevInfo d = device_info();
   if (!d.ok) return JF_ERR_DEVICE;
-  return cuda_status(jf::launch_quantize_granular(x, int(dt), rows, cols, int(g), q, s, d.status, d.sm_count,
+  return cuda_status(jf::launch_quantize_granular(x, int(dt), rows, cols, int(g), q, s,
+                                                   plain_loads_forced() ? nullptr : d.status, d.sm_count,
                                                   static_cast<cudaStream_t>(stream)));
 }
 

@@ -10,7 +10,8 @@ namespace jf {
 // The driver's cuTensorMapEncodeTiled (null if the driver does not provide it).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
-// `status`: the device status word, raised when a bounded wait in the kernel runs out.
+// `status`: the device status word, raised when a bounded wait in the kernel runs out; null selects
+// the plain-load kernel (no TMA staging, no waits).
 cudaError_t launch_quantize(const void* x, int dtype, int64_t R, int64_t C, int8_t* q, float* s,
                             unsigned int* status, int sm_count, cudaStream_t st);
 cudaError_t launch_dequantize(const int8_t* q, const float* s, int64_t R, int64_t C, void* y, int dtype,

@@ -1,5 +1,7 @@
 """GPU parity of the memory-bound per-block kernels against the CPU oracle:
 quantize (a1), dequantize (a2), GELU_i8 (a6), LayerNorm_i8 (a7)."""
+import zlib
+
 import numpy as np
 import pytest
 import torch
@@ -18,10 +20,15 @@ def _quant_gpu(x_dev):
     return host(t.q), host(t.s)
 
 
-@pytest.mark.parametrize("shape", [(32, 32), (96, 160), (256, 256), (64, 4096)])
+@pytest.mark.parametrize("path", ["tma", "plain"])
+@pytest.mark.parametrize("shape", [(32, 32), (96, 160), (256, 256), (64, 4096), (544, 96)])
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
-def test_quantize_bit_exact(shape, dtype):
-    rng = np.random.default_rng(hash((shape, dtype)) % 2 ** 31)
+def test_quantize_bit_exact(shape, dtype, path, monkeypatch):
+    """Both quantizer kernels: TMA-staged tiles (the default) and plain loads (JF_PLAIN_LOADS=1),
+    including odd block-column counts (the last tile's second block lies past the last column)."""
+    if path == "plain":
+        monkeypatch.setenv("JF_PLAIN_LOADS", "1")
+    rng = np.random.default_rng(zlib.crc32(f"{shape} {dtype}".encode()))  # stable across processes
     x = S.activation(rng, shape[0], shape[1], max(1, shape[1] // 100), 100.0)
     if dtype == "f32":
         xd, xh = dev_f32(x), x
