@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(32 * kGeluWarps, 3) gelu_i8_kernel(const int8_
                                                                     int64_t C, int8_t* __restrict__ qo,
                                                                     float* __restrict__ so) {
   __shared__ float table[kGeluWarps][2][256];
-  __shared__ __align__(16) uint8_t codes[kGeluWarps][2][256];
+  __shared__ __align__(256) uint8_t codes[kGeluWarps][2][256];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int64_t nbc = C >> 5;
   const int64_t npc = (nbc + 1) >> 1;   // block pairs per block row
@@ -365,13 +365,21 @@ __global__ void __launch_bounds__(32 * kGeluWarps, 3) gelu_i8_kernel(const int8_
       if (r0 == 0 && (vc & 1) == 0 && active) so[b0 + half] = __fdiv_rn(amax, kQMax);
     }
     __syncwarp();
+    const uint32_t cbase = smem_u32(ctab);  // 256-byte aligned: its low byte is zero
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
       const uint32_t w[4] = {a[t].x ^ 0x80808080u, a[t].y ^ 0x80808080u, a[t].z ^ 0x80808080u, a[t].w ^ 0x80808080u};
       uint32_t o[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        o[i] = pack4(ctab[w[i] & 0xFFu], ctab[(w[i] >> 8) & 0xFFu], ctab[(w[i] >> 16) & 0xFFu], ctab[w[i] >> 24]);
+      for (int i = 0; i < 4; ++i) {
+        uint32_t c[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t addr = __byte_perm(w[i], cbase, 0x7650 | k);  // byte k of w over the table base
+          asm volatile("ld.shared.u8 %0, [%1];" : "=r"(c[k]) : "r"(addr) : "memory");
+        }
+        o[i] = pack4(c[0], c[1], c[2], c[3]);
+      }
       if (active) *reinterpret_cast<uint4*>(qo + off + int64_t(t) * 8 * C) = make_uint4(o[0], o[1], o[2], o[3]);
     }
     __syncwarp();  // the tables are rewritten for the next pair only after every lane has read them
