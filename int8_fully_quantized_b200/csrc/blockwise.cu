@@ -281,7 +281,9 @@ __global__ void __launch_bounds__(256, 4) dequantize_kernel(const int8_t* __rest
 //      |GELU(x)| < 0.17 for x < 0, so when GELU(qmax s) >= 0.17 (qmax: the largest code, a bytewise
 //      integer max) it is the absmax; otherwise (rare) the lanes take the max over their lookups;
 //   3. code table: the quantized code of every table value (256 per block, the same rule as
-//      everywhere), so that each element costs one byte lookup.
+//      everywhere), so that each element costs one byte lookup; a table starts on a 256-byte
+//      boundary, so one `prmt` of the input word and the table's shared-memory address forms the
+//      address of an element's entry.
 // ---------------------------------------------------------------------------------------------
 constexpr int kGeluWarps = 8;
 constexpr float kGeluNegBound = 0.17f;  // > max |GELU(x)| over x < 0 (0.16997 at x = -0.7518)
