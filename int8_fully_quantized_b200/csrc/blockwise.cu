@@ -318,12 +318,15 @@ __global__ void __launch_bounds__(32 * kGeluWarps, 3) gelu_i8_kernel(const int8_
       float* tw = table[wib][tb];
       const float sc = (tb == 0 || has1) ? __ldg(s + b0 + tb) : 0.0f;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int m = k + 16 * j;                      // |code| 0..127
-        const float x = float(m) * sc;
-        const float e = erfc_nonneg(x * 0.70710678118654752440f);
-        tw[128 - m] = -0.5f * x * e;                   // code -m
-        tw[128 + m] = 0.5f * x * (2.0f - e);           // code +m (for m = 0 this +0 is the entry kept)
+      for (int j = 0; j < 8; j += 2) {
+        const int m0 = k + 16 * j, m1 = m0 + 16;       // |code| 0..127, two per packed erfc
+        const float x0 = float(m0) * sc, x1 = float(m1) * sc;
+        float e0, e1;
+        erfc_nonneg_x2(x0 * 0.70710678118654752440f, x1 * 0.70710678118654752440f, e0, e1);
+        tw[128 - m0] = -0.5f * x0 * e0;                // code -m
+        tw[128 + m0] = 0.5f * x0 * (2.0f - e0);        // code +m (for m = 0 this +0 is the entry kept)
+        tw[128 - m1] = -0.5f * x1 * e1;
+        tw[128 + m1] = 0.5f * x1 * (2.0f - e1);
       }
       if (k == 0) tw[0] = -0.5f * (128.0f * sc) * erfc_nonneg(128.0f * sc * 0.70710678118654752440f);  // code -128
     }
