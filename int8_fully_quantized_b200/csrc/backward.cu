@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(kLnbThreads, 2) layernorm_i8_bwd_kernel(
       const int8_t* xrow = xstrip + int64_t(rw) * H;
       const int8_t* drow = dstrip + int64_t(rw) * H;
       double sum_x = 0.0, sum_xx = 0.0, sum_g = 0.0, sum_gx = 0.0;
-      constexpr int kUnroll = 4;  // 16-byte chunks of each tensor a lane keeps in flight
+      constexpr int kUnroll = 2;  // 16-byte chunks of each tensor a lane keeps in flight (4 and 8: slower)
       for (int64_t ch0 = lane; ch0 < (H >> 4); ch0 += 32 * kUnroll) {
         uint4 av[kUnroll], dv[kUnroll];
         float scx[kUnroll], scd[kUnroll];
