@@ -292,7 +292,8 @@ __global__ void __launch_bounds__(32 * kGeluWarps, 3) gelu_i8_kernel(const int8_
                                                                     const float* __restrict__ s, int64_t R,
                                                                     int64_t C, int8_t* __restrict__ qo,
                                                                     float* __restrict__ so) {
-  __shared__ float table[kGeluWarps][2][256];
+  // both tables are indexed by the code's raw byte (q & 0xFF): the lookups use the input bytes as they are
+  __shared__ __align__(16) float table[kGeluWarps][2][256];
   __shared__ __align__(256) uint8_t codes[kGeluWarps][2][256];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int64_t nbc = C >> 5;
@@ -313,7 +314,7 @@ __global__ void __launch_bounds__(32 * kGeluWarps, 3) gelu_i8_kernel(const int8_
     uint4 a[4];
 #pragma unroll
     for (int t = 0; t < 4; ++t) a[t] = active ? ld_stream_v4(q + off + int64_t(t) * 8 * C) : make_uint4(0u, 0u, 0u, 0u);
-    // 1. value tables (index = code + 128)
+    // 1. value tables (index = the code's raw byte: +m at m, -m at 256 - m, -128 at 128)
     {
       float* tw = table[wib][tb];
       const float sc = (tb == 0 || has1) ? __ldg(s + b0 + tb) : 0.0f;
@@ -323,12 +324,12 @@ __global__ void __launch_bounds__(32 * kGeluWarps, 3) gelu_i8_kernel(const int8_
         const float x0 = float(m0) * sc, x1 = float(m1) * sc;
         float e0, e1;
         erfc_nonneg_x2(x0 * 0.70710678118654752440f, x1 * 0.70710678118654752440f, e0, e1);
-        tw[128 - m0] = -0.5f * x0 * e0;                // code -m
-        tw[128 + m0] = 0.5f * x0 * (2.0f - e0);        // code +m (for m = 0 this +0 is the entry kept)
-        tw[128 - m1] = -0.5f * x1 * e1;
-        tw[128 + m1] = 0.5f * x1 * (2.0f - e1);
+        tw[(128 - m0) ^ 0x80] = -0.5f * x0 * e0;       // code -m
+        tw[m0] = 0.5f * x0 * (2.0f - e0);              // code +m (for m = 0 this +0 is the entry kept)
+        tw[(128 - m1) ^ 0x80] = -0.5f * x1 * e1;
+        tw[m1] = 0.5f * x1 * (2.0f - e1);
       }
-      if (k == 0) tw[0] = -0.5f * (128.0f * sc) * erfc_nonneg(128.0f * sc * 0.70710678118654752440f);  // code -128
+      if (k == 0) tw[128] = -0.5f * (128.0f * sc) * erfc_nonneg(128.0f * sc * 0.70710678118654752440f);  // code -128
     }
     // 2. block absmax: the largest code of the lane's block (bytewise signed max), then its GELU
     uint32_t mx = 0x80808080u;
@@ -340,12 +341,12 @@ __global__ void __launch_bounds__(32 * kGeluWarps, 3) gelu_i8_kernel(const int8_
     qmax = max(qmax, __shfl_xor_sync(0xffffffffu, qmax, 8));
     qmax = max(qmax, __shfl_xor_sync(0xffffffffu, qmax, 16));
     __syncwarp();
-    float amax = tab[qmax + 128];
+    float amax = tab[qmax & 0xFF];
     if (__any_sync(0xffffffffu, !(amax >= kGeluNegBound))) {
       float m = 0.0f;
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        const uint32_t w[4] = {a[t].x ^ 0x80808080u, a[t].y ^ 0x80808080u, a[t].z ^ 0x80808080u, a[t].w ^ 0x80808080u};
+        const uint32_t w[4] = {a[t].x, a[t].y, a[t].z, a[t].w};
 #pragma unroll
         for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(tab[(w[i >> 2] >> (8 * (i & 3))) & 0xFFu]));
       }
@@ -355,25 +356,29 @@ __global__ void __launch_bounds__(32 * kGeluWarps, 3) gelu_i8_kernel(const int8_
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
       amax = m;
     }
-    // 3. code tables: lane k of each half quantizes entries k + 16 i of its block's table (consecutive
-    //    lanes touch consecutive words: no shared-memory bank conflicts)
+    // 3. code tables: lane k of each half quantizes the four consecutive entries 4k + 64 j .. + 3 of its
+    //    block's table (16-byte loads, one 4-byte store of four codes); the second half takes its j in
+    //    the order j + 1, so that in each store the two halves' words fall in different banks
     {
       const float amax_tb = __shfl_sync(0xffffffffu, amax, tb == 0 ? 0 : 2);  // lane 0: block 0, lane 2: block 1
       const BlockQuant bt = block_quant(amax_tb);
       float v[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] = table[wib][tb][k + 16 * i];
+      for (int j = 0; j < 4; ++j) {
+        const float4 f = *reinterpret_cast<const float4*>(&table[wib][tb][4 * k + 64 * ((j + tb) & 3)]);
+        v[4 * j] = f.x; v[4 * j + 1] = f.y; v[4 * j + 2] = f.z; v[4 * j + 3] = f.w;
+      }
       uint32_t o[4];
       quant_pack<16>(v, bt, o);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) codes[wib][tb][k + 16 * i] = uint8_t(o[i >> 2] >> (8 * (i & 3)));
+      for (int j = 0; j < 4; ++j) *reinterpret_cast<uint32_t*>(&codes[wib][tb][4 * k + 64 * ((j + tb) & 3)]) = o[j];
       if (r0 == 0 && (vc & 1) == 0 && active) so[b0 + half] = __fdiv_rn(amax, kQMax);
     }
     __syncwarp();
     const uint32_t cbase = smem_u32(ctab);  // 256-byte aligned: its low byte is zero
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
-      const uint32_t w[4] = {a[t].x ^ 0x80808080u, a[t].y ^ 0x80808080u, a[t].z ^ 0x80808080u, a[t].w ^ 0x80808080u};
+      const uint32_t w[4] = {a[t].x, a[t].y, a[t].z, a[t].w};
       uint32_t o[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
