@@ -43,16 +43,17 @@ __global__ void __launch_bounds__(32 * kGeluBwdWarps, 3) gelu_i8_bwd_kernel(
     const uint4 a1 = ld_stream_v4(xq + off + 16 * C);
     const uint4 d0 = ld_stream_v4(dq + off);
     const uint4 d1 = ld_stream_v4(dq + off + 16 * C);
-    // table[u] = GELU'(fp32(u - 128) * sx) for the code u - 128; one evaluation serves m and -m
+    // tab[b] = GELU'(fp32(q) * sx) for the code q whose raw byte is b (+m at m, -m at 256 - m, -128 at
+    // 128), so the lookups use the input bytes as they are; one evaluation serves m and -m
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int m = lane + 32 * j;  // |code| 0..127
       float gp, gn;
       gelu_grad_pair_f32(float(m) * sx, gp, gn);
-      tab[128 + m] = gp;
-      if (m != 0) tab[128 - m] = gn;
+      tab[m] = gp;
+      if (m != 0) tab[256 - m] = gn;
     }
-    if (lane == 0) tab[0] = gelu_grad_f32(-128.0f * sx);  // code -128
+    if (lane == 0) tab[128] = gelu_grad_f32(-128.0f * sx);  // code -128
     __syncwarp();
     const uint32_t wx[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
     const uint32_t wd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
@@ -60,7 +61,7 @@ __global__ void __launch_bounds__(32 * kGeluBwdWarps, 3) gelu_i8_bwd_kernel(
     float m = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const uint32_t u = wx[i] ^ 0x80808080u;  // code + 128 in each byte
+      const uint32_t u = wx[i];  // raw code bytes
       float g[4];
       i8x4_to_f32(wd[i], g);
 #pragma unroll
