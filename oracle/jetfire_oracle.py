@@ -45,7 +45,7 @@ __all__ = [
     "dequantize_block", "dequantize", "block_scale_grid", "linear_fwd", "linear_fwd_gelu", "linear_dgrad", "linear_wgrad",
     "requantize", "gelu_i8", "layernorm_i8", "gelu_f64", "quantization_mse", "gelu_grad_f64",
     "gelu_i8_bwd", "layernorm_i8_bwd", "E4M3_MAX", "e4m3_encode", "e4m3_decode", "mx_quantize",
-    "mx_dequantize", "mx_linear_fwd",
+    "mx_dequantize", "mx_linear_fwd", "quantize_block_rowstats", "rowstats_moments",
 ]
 
 
@@ -94,6 +94,32 @@ def quantize(x: np.ndarray, block_rows: int, block_cols: int):
 def quantize_block(x: np.ndarray):
     """Jetfire per-block quantizer: 32x32 blocks. Input fp32 (bf16/fp16 widened exactly first)."""
     return quantize(x, BLOCK, BLOCK)
+
+
+def quantize_block_rowstats(x: np.ndarray):
+    """f1, second half: the per-block quantizer that also hands LayerNorm_i8 the row statistics of
+    its output (the summary, "Approach": quantization on-chip, here carried one step further so that
+    LayerNorm needs no pass of its own over its input to find each row's mean and variance).
+
+    Returns (q, s, stats) with q, s as quantize_block and stats int64 [R, C/32, 2]: for row r and
+    block column J, stats[r, J] = (sum of q[r, j], sum of q[r, j]^2) over the block's 32 columns.
+    With x = q * s, the row's sum is sum_J s[r/32, J] * stats[r, J, 0] and its sum of squares
+    sum_J s[r/32, J]^2 * stats[r, J, 1] (exact products, as the integer sums are exact)."""
+    q, s = quantize_block(x)
+    R, C = q.shape
+    qb = q.astype(np.int64).reshape(R, C // BLOCK, BLOCK)
+    stats = np.stack([qb.sum(axis=2), (qb * qb).sum(axis=2)], axis=2)
+    return q, s, stats
+
+
+def rowstats_moments(stats: np.ndarray, s: np.ndarray, H: int):
+    """Mean and biased variance of each row of x = q * s from quantize_block_rowstats' sums, in fp64:
+    mean = sum_J s S1 / H, var = sum_J s^2 S2 / H - mean^2 (clamped at 0). Returns ([R], [R])."""
+    st = np.asarray(stats, np.float64)
+    sr = np.repeat(np.asarray(s, np.float64), BLOCK, axis=0)  # [R, C/32]: the scale of row r's blocks
+    mean = (sr * st[:, :, 0]).sum(axis=1) / H
+    var = np.maximum((sr * sr * st[:, :, 1]).sum(axis=1) / H - mean * mean, 0.0)
+    return mean, var
 
 
 def block_scale_grid(s: np.ndarray, block_rows: int = BLOCK, block_cols: int = BLOCK) -> np.ndarray:

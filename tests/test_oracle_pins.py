@@ -606,3 +606,35 @@ def test_mx_linear_fwd_exact_small_integers():
     assert np.array_equal(O.e4m3_decode(Aq), A) and np.array_equal(O.e4m3_decode(Bq), B)
     y = O.mx_linear_fwd(Aq, As, Bq, Bs)
     assert np.array_equal(y.astype(np.float64), (A.astype(np.int64) @ B.astype(np.int64).T) * 2.0)
+
+
+def test_quantize_rowstats_hand_worked_and_invariants():
+    """f1 row statistics: a hand-worked block whose scale is exactly 1 (so q = x), then invariants on
+    random outlier activations (block sums add up to the row sums taken over the whole row, the
+    Cauchy-Schwarz bound per block) and the moments against numpy's of x = q s."""
+    x = np.zeros((32, 64), np.float32)
+    for r in range(32):
+        x[r, :32] = r - 16          # block (0, 0): row r constant r - 16 ...
+    x[0, 5] = 127.0                 # ... except one 127, which makes s = 127 / 127 = 1
+    x[:, 32:] = -3.0                # block (0, 1): all -3, absmax 3, s = 3/127, q = -127
+    q, s, st = O.quantize_block_rowstats(x)
+    assert s[0, 0] == 1.0 and np.array_equal(q[:, :32], x[:, :32].astype(np.int8))
+    # by hand: row 0 holds 31 codes -16 and one 127; row r >= 1 holds 32 codes r - 16
+    assert st[0, 0, 0] == 31 * -16 + 127 == -369 and st[0, 0, 1] == 31 * 256 + 16129 == 24065
+    for r in range(1, 32):
+        assert st[r, 0, 0] == 32 * (r - 16) and st[r, 0, 1] == 32 * (r - 16) ** 2
+    assert np.all(st[:, 1, 0] == -127 * 32) and np.all(st[:, 1, 1] == 127 * 127 * 32)
+
+    rng = np.random.default_rng(91)
+    xr = S.activation(rng, 96, 160, 2, 50.0)
+    q, s, st = O.quantize_block_rowstats(xr)
+    qq, ss = O.quantize_block(xr)
+    assert np.array_equal(q, qq) and np.array_equal(s, ss)
+    q64 = q.astype(np.int64)
+    assert np.array_equal(st[:, :, 0].sum(axis=1), q64.sum(axis=1))
+    assert np.array_equal(st[:, :, 1].sum(axis=1), (q64 * q64).sum(axis=1))
+    assert np.all(st[:, :, 0] ** 2 <= 32 * st[:, :, 1]) and np.all(np.abs(st[:, :, 0]) <= 32 * 127)
+    mean, var = O.rowstats_moments(st, s, xr.shape[1])
+    xe = q.astype(np.float64) * np.repeat(np.repeat(s.astype(np.float64), 32, axis=0), 32, axis=1)
+    assert np.allclose(mean, xe.mean(axis=1), rtol=1e-12, atol=1e-15)
+    assert np.allclose(var, xe.var(axis=1), rtol=1e-9, atol=1e-15)
