@@ -101,6 +101,18 @@ JF_API int jf_quantize_block(const void* x, jf_dtype dt, int64_t rows, int64_t c
                       void* stream);
 
 /*
+ * f1 (second half). jf_quantize_block that also writes the row statistics LayerNorm_i8 needs of
+ * its input (summary, "Approach": quantization on-chip; here the LayerNorm's row sums move into the
+ * op that produces its input, so the LayerNorm needs no pass of its own to find them).
+ *   stats  device int32 [rows][cols/32][2], 8-byte aligned (output): for row r and block column J,
+ *          (sum of q[r, j], sum of q[r, j]^2) over the block's 32 columns (exact integers).
+ * q and s are identical to jf_quantize_block's. Errors as jf_quantize_block, plus JF_ERR_NULL /
+ * JF_ERR_ALIGN / JF_ERR_ALIAS for stats.
+ */
+JF_API int jf_quantize_block_rowstats(const void* x, jf_dtype dt, int64_t rows, int64_t cols, int8_t* q, float* s,
+                                      int32_t* stats, void* stream);
+
+/*
  * a2. Dequantization y = fp32(q) * s, rounded to nearest even into `dt` ("Fp8 vs int8" page).
  *   q, s  the quantized tensor (device, layout as above)
  *   y     device, [rows, cols] of dtype `dt`, 16-byte aligned (output); bit-exact.
@@ -164,6 +176,17 @@ JF_API int jf_gelu_i8(jf_cqtensor X, jf_qtensor Y, void* stream);
  */
 JF_API int jf_layernorm_i8(jf_cqtensor X, const float* gamma, const float* beta, float eps, jf_qtensor Y,
                     void* stream);
+
+/*
+ * f1 (second half). jf_layernorm_i8 with each row's mean and biased variance formed from `stats`,
+ * the row statistics jf_quantize_block_rowstats wrote for X (mean = sum_J s * S1 / H, mean square
+ * = sum_J s^2 * S2 / H, in fp64), so X is read once. The caller passes the stats of this X; the
+ * result is then LayerNorm_i8 of X (the row sums are the same numbers, added in another order).
+ *   stats  device int32 [rows][cols/32][2], 8-byte aligned.
+ * Errors as jf_layernorm_i8, plus JF_ERR_NULL / JF_ERR_ALIGN / JF_ERR_ALIAS for stats.
+ */
+JF_API int jf_layernorm_i8_rowstats(jf_cqtensor X, const int32_t* stats, const float* gamma, const float* beta,
+                                    float eps, jf_qtensor Y, void* stream);
 
 /*
  * f2. Backward of GELU_i8 (summary, "Approach": the backward pass keeps the INT8 data flow too).

@@ -27,6 +27,7 @@ __all__ = [
     # C ABI, one wrapper per entry point
     "jf_quantize_block", "jf_dequantize_block", "jf_linear_fwd", "jf_linear_fwd_gelu", "jf_linear_dgrad",
     "jf_linear_wgrad", "jf_gelu_i8", "jf_layernorm_i8", "jf_gelu_i8_bwd", "jf_layernorm_i8_bwd",
+    "jf_quantize_block_rowstats", "jf_layernorm_i8_rowstats", "quantize_block_rowstats", "layernorm_i8_rowstats",
     "jf_layernorm_i8_bwd_workspace_bytes", "jf_layernorm_i8_bwd_noalloc", "jf_quantize_granular",
     "jf_dequantize_granular", "jf_quantization_error", "jf_granular_scale_count", "jf_mx_quantize",
     "jf_mx_linear_fwd", "jf_selftest_wait_timeout", "jf_strerror",
@@ -42,7 +43,7 @@ GRANULARITY = {"block": 0, "token": 1, "channel": 2, "tensor": 3}
 _DTYPES = {torch.float32: JF_F32, torch.bfloat16: JF_BF16, torch.float16: JF_F16}
 
 EXPORTED_SYMBOLS = (
-    "jf_quantize_block", "jf_dequantize_block", "jf_linear_fwd", "jf_linear_fwd_gelu", "jf_linear_dgrad",
+    "jf_quantize_block", "jf_quantize_block_rowstats", "jf_layernorm_i8_rowstats", "jf_dequantize_block", "jf_linear_fwd", "jf_linear_fwd_gelu", "jf_linear_dgrad",
     "jf_linear_wgrad",
     "jf_gelu_i8", "jf_layernorm_i8", "jf_gelu_i8_bwd", "jf_layernorm_i8_bwd", "jf_layernorm_i8_bwd_workspace_bytes",
     "jf_layernorm_i8_bwd_noalloc", "jf_quantize_granular", "jf_dequantize_granular", "jf_quantization_error",
@@ -89,6 +90,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.jf_linear_fwd_gelu.argtypes = [_CQ, _CQ, _Q, _Q, vp]
     lib.jf_gelu_i8.argtypes = [_CQ, _Q, vp]
     lib.jf_layernorm_i8.argtypes = [_CQ, vp, vp, ctypes.c_float, _Q, vp]
+    lib.jf_quantize_block_rowstats.argtypes = [vp, i32, i64, i64, vp, vp, vp, vp]
+    lib.jf_layernorm_i8_rowstats.argtypes = [_CQ, vp, vp, vp, ctypes.c_float, _Q, vp]
     lib.jf_gelu_i8_bwd.argtypes = [_CQ, _CQ, _Q, vp]
     lib.jf_layernorm_i8_bwd.argtypes = [_CQ, _CQ, vp, ctypes.c_float, _Q, vp, vp, vp, i64, vp]
     lib.jf_layernorm_i8_bwd_workspace_bytes.argtypes = [i64, i64]
@@ -169,6 +172,13 @@ def jf_quantize_block(x: torch.Tensor, q: torch.Tensor, s: torch.Tensor, stream=
                                  _stream(stream)), "jf_quantize_block")
 
 
+def jf_quantize_block_rowstats(x: torch.Tensor, q: torch.Tensor, s: torch.Tensor, stats: torch.Tensor,
+                               stream=None) -> None:
+    lib = load_library()
+    _check(lib.jf_quantize_block_rowstats(_ptr(x), _DTYPES[x.dtype], x.shape[0], x.shape[1], _ptr(q), _ptr(s),
+                                          _ptr(stats), _stream(stream)), "jf_quantize_block_rowstats")
+
+
 def jf_dequantize_block(q: torch.Tensor, s: torch.Tensor, y: torch.Tensor, stream=None) -> None:
     lib = load_library()
     if y.dtype not in _DTYPES:
@@ -213,6 +223,13 @@ def jf_layernorm_i8(X: QTensor, gamma: torch.Tensor, beta: torch.Tensor, eps: fl
     lib = load_library()
     _check(lib.jf_layernorm_i8(_cq(X), _ptr(gamma), _ptr(beta), ctypes.c_float(eps), _q(Y, X.rows, X.cols),
                                _stream(stream)), "jf_layernorm_i8")
+
+
+def jf_layernorm_i8_rowstats(X: QTensor, stats: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor, eps: float,
+                             Y: QTensor, stream=None) -> None:
+    lib = load_library()
+    _check(lib.jf_layernorm_i8_rowstats(_cq(X), _ptr(stats), _ptr(gamma), _ptr(beta), ctypes.c_float(eps),
+                                        _q(Y, X.rows, X.cols), _stream(stream)), "jf_layernorm_i8_rowstats")
 
 
 def jf_gelu_i8_bwd(X: QTensor, dY: QTensor, dX: QTensor, stream=None) -> None:
@@ -397,4 +414,21 @@ def layernorm_i8_bwd(X: QTensor, dY: QTensor, gamma: torch.Tensor, eps: float = 
 def layernorm_i8(X: QTensor, gamma: torch.Tensor, beta: torch.Tensor, eps: float = 1e-5, stream=None) -> QTensor:
     Y = empty_qtensor(X.rows, X.cols, X.q.device)
     jf_layernorm_i8(X, gamma, beta, eps, Y, stream)
+    return Y
+
+
+
+def quantize_block_rowstats(x: torch.Tensor, stream=None):
+    """(QTensor, stats): the per-block quantization of x and, per row and block, the int32 sums of q
+    and q^2 ([rows, cols/32, 2]) that layernorm_i8_rowstats takes in place of a pass over the codes."""
+    out = empty_qtensor(x.shape[0], x.shape[1], x.device)
+    stats = torch.empty((x.shape[0], x.shape[1] // 32, 2), dtype=torch.int32, device=x.device)
+    jf_quantize_block_rowstats(x, out.q, out.s, stats, stream)
+    return out, stats
+
+
+def layernorm_i8_rowstats(X: QTensor, stats: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor,
+                          eps: float = 1e-5, stream=None) -> QTensor:
+    Y = empty_qtensor(X.rows, X.cols, X.q.device)
+    jf_layernorm_i8_rowstats(X, stats, gamma, beta, eps, Y, stream)
     return Y

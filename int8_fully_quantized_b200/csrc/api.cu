@@ -162,21 +162,40 @@ int gemm_call(int mode, const jf_cqtensor& A, const jf_cqtensor& B, const jf_qte
 
 extern "C" {
 
-int jf_quantize_block(const void* x, jf_dtype dt, int64_t rows, int64_t cols, int8_t* q, float* s,
-                      void* stream) {
+// Bytes of the row statistics of a [rows, cols] tensor: int32 [rows][cols/32][2].
+inline int64_t statbytes(int64_t rows, int64_t cols) { return rows * (cols / 32) * 2 * 4; }
+
+static int quantize_impl(const void* x, jf_dtype dt, int64_t rows, int64_t cols, int8_t* q, float* s,
+                         int32_t* stats, bool want_stats, void* stream) {
   if (dt != JF_F32 && dt != JF_BF16 && dt != JF_F16) return JF_ERR_DTYPE;
   if (!dims_ok(rows, cols)) return JF_ERR_SHAPE;
   if (rows == 0 || cols == 0) return JF_OK;
-  if (x == nullptr || q == nullptr || s == nullptr) return JF_ERR_NULL;
-  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(s, 4)) return JF_ERR_ALIGN;
+  if (x == nullptr || q == nullptr || s == nullptr || (want_stats && stats == nullptr)) return JF_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(q, 16) || !aligned(s, 4) || (want_stats && !aligned(stats, 8))) return JF_ERR_ALIGN;
   const int64_t nx = rows * cols * elem_size(dt);
   if (overlap(q, rows * cols, x, nx) || overlap(s, sbytes(rows, cols), x, nx) ||
       overlap(q, rows * cols, s, sbytes(rows, cols)))
     return JF_ERR_ALIAS;
+  if (want_stats) {
+    const int64_t nst = statbytes(rows, cols);
+    if (overlap(stats, nst, x, nx) || overlap(stats, nst, q, rows * cols) || overlap(stats, nst, s, sbytes(rows, cols)))
+      return JF_ERR_ALIAS;
+  }
   const DevInfo d = device_info();
   if (!d.ok) return JF_ERR_DEVICE;
-  return cuda_status(jf::launch_quantize(x, int(dt), rows, cols, q, s, plain_loads_forced() ? nullptr : d.status,
-                                          d.sm_count, static_cast<cudaStream_t>(stream)));
+  return cuda_status(jf::launch_quantize(x, int(dt), rows, cols, q, s, want_stats ? stats : nullptr,
+                                          plain_loads_forced() ? nullptr : d.status, d.sm_count,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+int jf_quantize_block(const void* x, jf_dtype dt, int64_t rows, int64_t cols, int8_t* q, float* s,
+                      void* stream) {
+  return quantize_impl(x, dt, rows, cols, q, s, nullptr, false, stream);
+}
+
+int jf_quantize_block_rowstats(const void* x, jf_dtype dt, int64_t rows, int64_t cols, int8_t* q, float* s,
+                               int32_t* stats, void* stream) {
+  return quantize_impl(x, dt, rows, cols, q, s, stats, true, stream);
 }
 
 int jf_dequantize_block(const int8_t* q, const float* s, int64_t rows, int64_t cols, void* y, jf_dtype dt,
@@ -233,24 +252,38 @@ int jf_gelu_i8(jf_cqtensor X, jf_qtensor Y, void* stream) {
   return cuda_status(jf::launch_gelu_i8(X.q, X.s, X.rows, X.cols, Y.q, Y.s, d.sm_count, static_cast<cudaStream_t>(stream)));
 }
 
-int jf_layernorm_i8(jf_cqtensor X, const float* gamma, const float* beta, float eps, jf_qtensor Y,
-                    void* stream) {
+static int layernorm_impl(jf_cqtensor X, const int32_t* stats, bool want_stats, const float* gamma,
+                          const float* beta, float eps, jf_qtensor Y, void* stream) {
   int st;
   if ((st = check_cq(X)) != JF_OK) return st;
   if ((st = check_q(Y, true)) != JF_OK) return st;
   if (X.rows != Y.rows || X.cols != Y.cols) return JF_ERR_SHAPE;
   if (X.rows == 0 || X.cols == 0) return JF_OK;
-  if (gamma == nullptr || beta == nullptr) return JF_ERR_NULL;
-  if (!aligned(gamma, 16) || !aligned(beta, 16)) return JF_ERR_ALIGN;
+  if (gamma == nullptr || beta == nullptr || (want_stats && stats == nullptr)) return JF_ERR_NULL;
+  if (!aligned(gamma, 16) || !aligned(beta, 16) || (want_stats && !aligned(stats, 8))) return JF_ERR_ALIGN;
   const int64_t nq = qbytes(X), ns = sbytes(X.rows, X.cols);
   if (overlap(Y.q, nq, X.q, nq) || overlap(Y.q, nq, X.s, ns) || overlap(Y.s, ns, X.q, nq) ||
       overlap(Y.s, ns, X.s, ns) || overlap(Y.q, nq, Y.s, ns) || overlap(Y.q, nq, gamma, X.cols * 4) ||
       overlap(Y.q, nq, beta, X.cols * 4) || overlap(Y.s, ns, gamma, X.cols * 4) || overlap(Y.s, ns, beta, X.cols * 4))
     return JF_ERR_ALIAS;
+  if (want_stats) {
+    const int64_t nst = statbytes(X.rows, X.cols);
+    if (overlap(Y.q, nq, stats, nst) || overlap(Y.s, ns, stats, nst)) return JF_ERR_ALIAS;
+  }
   const DevInfo d = device_info();
   if (!d.ok) return JF_ERR_DEVICE;
-  return cuda_status(
-      jf::launch_layernorm_i8(X.q, X.s, X.rows, X.cols, gamma, beta, eps, Y.q, Y.s, static_cast<cudaStream_t>(stream)));
+  return cuda_status(jf::launch_layernorm_i8(X.q, X.s, X.rows, X.cols, gamma, beta, eps, Y.q, Y.s,
+                                             want_stats ? stats : nullptr, static_cast<cudaStream_t>(stream)));
+}
+
+int jf_layernorm_i8(jf_cqtensor X, const float* gamma, const float* beta, float eps, jf_qtensor Y,
+                    void* stream) {
+  return layernorm_impl(X, nullptr, false, gamma, beta, eps, Y, stream);
+}
+
+int jf_layernorm_i8_rowstats(jf_cqtensor X, const int32_t* stats, const float* gamma, const float* beta, float eps,
+                             jf_qtensor Y, void* stream) {
+  return layernorm_impl(X, stats, true, gamma, beta, eps, Y, stream);
 }
 
 int jf_gelu_i8_bwd(jf_cqtensor X, jf_cqtensor dY, jf_qtensor dX, void* stream) {

@@ -32,9 +32,36 @@ namespace jf {
 // cleared), reduced over the 16 lanes of the lane's block, and the values are unpacked and quantized
 // eight at a time. When the number of block columns is odd the last pair holds one block.
 // ---------------------------------------------------------------------------------------------
+// f1 row statistics: for the group of eight codes w just quantized (VPG vectors of EPV codes; a vector
+// covers EPV consecutive columns of one row), the sums of q and q^2 over each vector's row of the
+// block, added over the HALF lanes that hold that row of the block (exact integers, |sum q| <= 4064,
+// sum q^2 <= 516128) and stored by the first of them as stats[row][block] = (sum q, sum q^2).
+template <int EPV, int VPG, int HALF>
+__device__ __forceinline__ void store_row_stats(const uint32_t (&w)[2], int* __restrict__ stats, int64_t row0,
+                                                int64_t rstep, int64_t nbc, int64_t bj, bool store) {
+#pragma unroll
+  for (int g = 0; g < VPG; ++g) {
+    int s1, s2;
+    if constexpr (EPV == 8) {
+      s1 = __dp4a(int(w[0]), 0x01010101, __dp4a(int(w[1]), 0x01010101, 0));
+      s2 = __dp4a(int(w[0]), int(w[0]), __dp4a(int(w[1]), int(w[1]), 0));
+    } else {
+      s1 = __dp4a(int(w[g]), 0x01010101, 0);
+      s2 = __dp4a(int(w[g]), int(w[g]), 0);
+    }
+#pragma unroll
+    for (int o = 1; o < HALF; o <<= 1) {
+      s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+      s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+    }
+    if (store) *reinterpret_cast<int2*>(stats + 2 * ((row0 + g * rstep) * nbc + bj)) = make_int2(s1, s2);
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256, 3) quantize_kernel(const T* __restrict__ x, int64_t R, int64_t C,
-                                                          int8_t* __restrict__ q, float* __restrict__ s) {
+                                                          int8_t* __restrict__ q, float* __restrict__ s,
+                                                          int* __restrict__ stats) {
   constexpr int EPV = Vec<T>::kElems;      // elements per 16-byte vector
   constexpr int VPR = 64 / EPV;            // vectors per tile row (= vectors per lane)
   constexpr int RSTEP = 32 / VPR;          // rows between a lane's vectors
@@ -80,6 +107,9 @@ __global__ void __launch_bounds__(256, 3) quantize_kernel(const T* __restrict__ 
       for (int g = 0; g < VPG; ++g) Vec<T>::unpack(raw[t + g], *reinterpret_cast<float(*)[EPV]>(v + g * EPV));
       uint32_t w[2];
       quant_pack<8>(v, bq, w);
+      if (stats != nullptr)
+        store_row_stats<EPV, VPG, HALF>(w, stats, bi * 32 + r0 + int64_t(t) * RSTEP, RSTEP, nbc, bj,
+                                        active && vc % HALF == 0);
       if (active) {
         if constexpr (EPV == 4) {
           *reinterpret_cast<uint32_t*>(dst + int64_t(t) * RSTEP * C) = w[0];
@@ -122,7 +152,8 @@ __host__ __device__ constexpr int qt_smem_bytes() { return QtCfg<T>::kWarps * Qt
 template <typename T>
 __global__ void __launch_bounds__(32 * QtCfg<T>::kWarps, 1) quantize_tma_kernel(const __grid_constant__ CUtensorMap map,
                                                                               int64_t R, int64_t C, int8_t* __restrict__ q,
-                                                                              float* __restrict__ s, unsigned int* status) {
+                                                                              float* __restrict__ s, int* __restrict__ stats,
+                                                                              unsigned int* status) {
   constexpr int EPV = Vec<T>::kElems;
   constexpr int VPR = 64 / EPV;
   constexpr int RSTEP = 32 / VPR;
@@ -205,6 +236,9 @@ __global__ void __launch_bounds__(32 * QtCfg<T>::kWarps, 1) quantize_tma_kernel(
       for (int g = 0; g < VPG; ++g) Vec<T>::unpack(raw[t + g], *reinterpret_cast<float(*)[EPV]>(v + g * EPV));
       uint32_t w[2];
       quant_pack<8>(v, bq, w);
+      if (stats != nullptr)
+        store_row_stats<EPV, VPG, HALF>(w, stats, bi * 32 + r0 + int64_t(t) * RSTEP, RSTEP, nbc, bj,
+                                        active && vc % HALF == 0);
       if (active) {
         if constexpr (EPV == 4) {
           *reinterpret_cast<uint32_t*>(dst + int64_t(t) * RSTEP * C) = w[0];
@@ -414,7 +448,8 @@ __global__ void __launch_bounds__(kLnThreads, 2) layernorm_i8_kernel(const int8_
                                                                   int64_t H, const float* __restrict__ gamma,
                                                                   const float* __restrict__ beta, float eps,
                                                                   int8_t* __restrict__ qo,
-                                                                  float* __restrict__ so) {
+                                                                  float* __restrict__ so,
+                                                                  const int* __restrict__ stats) {
   __shared__ float s_mean[32], s_rstd[32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t strip = blockIdx.x;
@@ -422,45 +457,72 @@ __global__ void __launch_bounds__(kLnThreads, 2) layernorm_i8_kernel(const int8_
   const int8_t* qs = q + strip * 32 * H;
   const float* ss = s + strip * nbc;
   const uint64_t keep = l2_policy_evict_last(), stream = l2_policy_evict_first();
-  for (int rw = warp; rw < 32; rw += kLnThreads / 32) {
-    const int8_t* row = qs + int64_t(rw) * H;
-    double sum = 0.0, sq = 0.0;
-    constexpr int kUnroll = 8;  // 16-byte chunks of the row a lane keeps in flight
-    for (int64_t ch0 = lane; ch0 < (H >> 4); ch0 += 32 * kUnroll) {
-      uint4 av[kUnroll];
-      float scv[kUnroll];
+  if (stats != nullptr) {
+    // f1: the row sums come with the input (the quantizer's exact integer sums per row and block):
+    // lane j adds blocks j, j + 32, ... of the row in fp64, then a fixed shuffle tree adds the lanes
+    for (int rw = warp; rw < 32; rw += kLnThreads / 32) {
+      const int2* st = reinterpret_cast<const int2*>(stats) + (strip * 32 + rw) * nbc;
+      double sum = 0.0, sq = 0.0;
+      for (int64_t J = lane; J < nbc; J += 32) {
+        const int2 v = __ldg(st + J);
+        const double sc = double(__ldg(ss + J));
+        sum = fma(sc, double(v.x), sum);
+        sq = fma(sc * sc, double(v.y), sq);
+      }
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int64_t ch = ch0 + 32 * u;
-        if (ch < (H >> 4)) {
-          av[u] = ld_v4_policy(row + ch * 16, keep);  // read again in phase 2: keep it in L2
-          scv[u] = __ldg(ss + (ch >> 1));
-        } else {
-          av[u] = make_uint4(0u, 0u, 0u, 0u);
-          scv[u] = 0.0f;
+      for (int o = 16; o > 0; o >>= 1) {
+        sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      }
+      if (lane == 0) {
+        const double mean = sum / double(H);
+        double var = sq / double(H) - mean * mean;
+        var = var > 0.0 ? var : 0.0;
+        s_mean[rw] = float(mean);
+        s_rstd[rw] = float(1.0 / sqrt(var + double(eps)));
+      }
+    }
+  } else {
+    for (int rw = warp; rw < 32; rw += kLnThreads / 32) {
+      const int8_t* row = qs + int64_t(rw) * H;
+      double sum = 0.0, sq = 0.0;
+      constexpr int kUnroll = 8;  // 16-byte chunks of the row a lane keeps in flight
+      for (int64_t ch0 = lane; ch0 < (H >> 4); ch0 += 32 * kUnroll) {
+        uint4 av[kUnroll];
+        float scv[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const int64_t ch = ch0 + 32 * u;
+          if (ch < (H >> 4)) {
+            av[u] = ld_v4_policy(row + ch * 16, keep);  // read again in phase 2: keep it in L2
+            scv[u] = __ldg(ss + (ch >> 1));
+          } else {
+            av[u] = make_uint4(0u, 0u, 0u, 0u);
+            scv[u] = 0.0f;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          // the 16 codes of a chunk share one block scale: their sum and sum of squares are exact
+          // integers (4-way byte dot products), scaled once in fp64
+          const int is = chunk_sum_i8(av[u]), iq = chunk_sumsq_i8(av[u]);
+          const double sc = double(scv[u]);
+          sum = fma(sc, double(is), sum);
+          sq = fma(sc * sc, double(iq), sq);
         }
       }
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        // the 16 codes of a chunk share one block scale: their sum and sum of squares are exact
-        // integers (4-way byte dot products), scaled once in fp64
-        const int is = chunk_sum_i8(av[u]), iq = chunk_sumsq_i8(av[u]);
-        const double sc = double(scv[u]);
-        sum = fma(sc, double(is), sum);
-        sq = fma(sc * sc, double(iq), sq);
+      for (int o = 16; o > 0; o >>= 1) {
+        sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        sq += __shfl_xor_sync(0xffffffffu, sq, o);
       }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      sq += __shfl_xor_sync(0xffffffffu, sq, o);
-    }
-    if (lane == 0) {
-      const double mean = sum / double(H);
-      double var = sq / double(H) - mean * mean;
-      var = var > 0.0 ? var : 0.0;
-      s_mean[rw] = float(mean);
-      s_rstd[rw] = float(1.0 / sqrt(var + double(eps)));
+      if (lane == 0) {
+        const double mean = sum / double(H);
+        double var = sq / double(H) - mean * mean;
+        var = var > 0.0 ? var : 0.0;
+        s_mean[rw] = float(mean);
+        s_rstd[rw] = float(1.0 / sqrt(var + double(eps)));
+      }
     }
   }
   __syncthreads();
@@ -536,7 +598,7 @@ static bool make_quant_map(CUtensorMap* m, const void* x, int dtype, int64_t R, 
 }
 
 template <typename T>
-static cudaError_t run_quantize_tma(const CUtensorMap& map, int64_t R, int64_t C, int8_t* q, float* s,
+static cudaError_t run_quantize_tma(const CUtensorMap& map, int64_t R, int64_t C, int8_t* q, float* s, int* stats,
                                     unsigned int* status, int sm_count, cudaStream_t st) {
   static unsigned long long attr_set = 0;  // one bit per device ordinal
   auto kern = quantize_tma_kernel<T>;
@@ -552,26 +614,26 @@ static cudaError_t run_quantize_tma(const CUtensorMap& map, int64_t R, int64_t C
   const int64_t npairs = (R / 32) * ((C / 32 + 1) / 2);
   int64_t grid = (npairs + QtCfg<T>::kWarps - 1) / QtCfg<T>::kWarps;
   if (grid > sm_count) grid = sm_count;
-  kern<<<int(grid), 32 * QtCfg<T>::kWarps, qt_smem_bytes<T>(), st>>>(map, R, C, q, s, status);
+  kern<<<int(grid), 32 * QtCfg<T>::kWarps, qt_smem_bytes<T>(), st>>>(map, R, C, q, s, stats, status);
   return cudaGetLastError();
 }
 
-cudaError_t launch_quantize(const void* x, int dtype, int64_t R, int64_t C, int8_t* q, float* s,
+cudaError_t launch_quantize(const void* x, int dtype, int64_t R, int64_t C, int8_t* q, float* s, int32_t* stats,
                             unsigned int* status, int sm_count, cudaStream_t st) {
   CUtensorMap map;
   if (status != nullptr && make_quant_map(&map, x, dtype, R, C)) {
-    if (dtype == 0) return run_quantize_tma<float>(map, R, C, q, s, status, sm_count, st);
-    if (dtype == 1) return run_quantize_tma<__nv_bfloat16>(map, R, C, q, s, status, sm_count, st);
-    return run_quantize_tma<__half>(map, R, C, q, s, status, sm_count, st);
+    if (dtype == 0) return run_quantize_tma<float>(map, R, C, q, s, stats, status, sm_count, st);
+    if (dtype == 1) return run_quantize_tma<__nv_bfloat16>(map, R, C, q, s, stats, status, sm_count, st);
+    return run_quantize_tma<__half>(map, R, C, q, s, stats, status, sm_count, st);
   }
   // no tensor map for this input (the driver refused it): plain loads
   const int grid = grid_for_blocks((R / 32) * ((C / 32 + 1) / 2), sm_count);  // one warp per block pair
   if (dtype == 0)
-    quantize_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), R, C, q, s);
+    quantize_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), R, C, q, s, stats);
   else if (dtype == 1)
-    quantize_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), R, C, q, s);
+    quantize_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), R, C, q, s, stats);
   else
-    quantize_kernel<__half><<<grid, 256, 0, st>>>(static_cast<const __half*>(x), R, C, q, s);
+    quantize_kernel<__half><<<grid, 256, 0, st>>>(static_cast<const __half*>(x), R, C, q, s, stats);
   return cudaGetLastError();
 }
 
@@ -595,8 +657,9 @@ cudaError_t launch_gelu_i8(const int8_t* q, const float* s, int64_t R, int64_t C
 }
 
 cudaError_t launch_layernorm_i8(const int8_t* q, const float* s, int64_t R, int64_t H, const float* gamma,
-                                const float* beta, float eps, int8_t* qo, float* so, cudaStream_t st) {
-  layernorm_i8_kernel<<<int(R / 32), kLnThreads, 0, st>>>(q, s, R, H, gamma, beta, eps, qo, so);
+                                const float* beta, float eps, int8_t* qo, float* so, const int32_t* stats,
+                                cudaStream_t st) {
+  layernorm_i8_kernel<<<int(R / 32), kLnThreads, 0, st>>>(q, s, R, H, gamma, beta, eps, qo, so, stats);
   return cudaGetLastError();
 }
 

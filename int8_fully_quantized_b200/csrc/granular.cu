@@ -261,7 +261,7 @@ static cudaError_t quantize_granular_t(const T* x, int64_t R, int64_t C, int g, 
 
 cudaError_t launch_quantize_granular(const void* x, int dtype, int64_t R, int64_t C, int g, int8_t* q, float* s,
                                      unsigned int* status, int sm_count, cudaStream_t st) {
-  if (g == kGranBlock) return launch_quantize(x, dtype, R, C, q, s, status, sm_count, st);
+  if (g == kGranBlock) return launch_quantize(x, dtype, R, C, q, s, nullptr, status, sm_count, st);
   if (dtype == 0) return quantize_granular_t(static_cast<const float*>(x), R, C, g, q, s, sm_count, st);
   if (dtype == 1) return quantize_granular_t(static_cast<const __nv_bfloat16*>(x), R, C, g, q, s, sm_count, st);
   return quantize_granular_t(static_cast<const __half*>(x), R, C, g, q, s, sm_count, st);

@@ -11,8 +11,9 @@ namespace jf {
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 // `status`: the device status word, raised when a bounded wait in the kernel runs out; null selects
-// the plain-load kernel (no TMA staging, no waits).
-cudaError_t launch_quantize(const void* x, int dtype, int64_t R, int64_t C, int8_t* q, float* s,
+// the plain-load kernel (no TMA staging, no waits). `stats` (optional, int32 [R][C/32][2]): per row
+// and block, the sums of q and q^2 (what LayerNorm_i8 needs of its input rows).
+cudaError_t launch_quantize(const void* x, int dtype, int64_t R, int64_t C, int8_t* q, float* s, int32_t* stats,
                             unsigned int* status, int sm_count, cudaStream_t st);
 cudaError_t launch_dequantize(const int8_t* q, const float* s, int64_t R, int64_t C, void* y, int dtype,
                               int sm_count, cudaStream_t st);
@@ -54,7 +55,8 @@ cudaError_t launch_layernorm_i8_bwd(const int8_t* xq, const float* xs, const int
                                     int64_t H, const float* gamma, float eps, int8_t* qo, float* so, float* part,
                                     float* dgamma, float* dbeta, cudaStream_t st);
 cudaError_t launch_layernorm_i8(const int8_t* q, const float* s, int64_t R, int64_t H, const float* gamma,
-                                const float* beta, float eps, int8_t* qo, float* so, cudaStream_t st);
+                                const float* beta, float eps, int8_t* qo, float* so, const int32_t* stats,
+                                cudaStream_t st);
 
 // Block-scaled INT8 GEMM: out[r, c] = sum over 32-blocks kb of the contraction axis of
 // fp32(sA(r/32, kb) * sB(c/32, kb)) * sum_{k in kb} A(r, k) B(c, k), re-quantized per 32x32 block.

@@ -118,6 +118,16 @@ def test_host_validation_rejects_bad_arguments(lib):
     # LayerNorm needs gamma/beta
     assert lib.jf_layernorm_i8(jf._CQ(1 << 20, 1 << 22, 32, 64), None, fake, ctypes.c_float(1e-5),
                                jf._Q(1 << 28, 1 << 30, 32, 64), None) == -1
+    # f1 row statistics: the stats buffer is required, 8-byte aligned and apart from the other buffers
+    assert lib.jf_quantize_block_rowstats(fake, 1, 32, 64, vp(1 << 22), vp(1 << 23), None, None) == -1
+    assert lib.jf_quantize_block_rowstats(fake, 1, 32, 64, vp(1 << 22), vp(1 << 23), vp((1 << 24) + 4), None) == -3
+    assert lib.jf_quantize_block_rowstats(fake, 1, 32, 64, vp(1 << 22), vp(1 << 23), vp((1 << 22) + 8), None) == -5
+    assert lib.jf_quantize_block_rowstats(fake, 1, 33, 64, vp(1 << 22), vp(1 << 23), vp(1 << 24), None) == -2
+    assert lib.jf_quantize_block_rowstats(None, 1, 0, 64, None, None, None, None) == 0
+    Xl, Yl = jf._CQ(1 << 20, 1 << 22, 32, 64), jf._Q(1 << 28, 1 << 30, 32, 64)
+    assert lib.jf_layernorm_i8_rowstats(Xl, None, fake, fake, ctypes.c_float(1e-5), Yl, None) == -1
+    assert lib.jf_layernorm_i8_rowstats(Xl, vp((1 << 24) + 4), fake, fake, ctypes.c_float(1e-5), Yl, None) == -3
+    assert lib.jf_layernorm_i8_rowstats(Xl, vp((1 << 28) + 16), fake, fake, ctypes.c_float(1e-5), Yl, None) == -5
 
 
 @pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-GPU behaviour")

@@ -221,3 +221,56 @@ def test_empty_inputs_are_noops():
     t = jf.quantize_block(z)
     assert t.q.shape == (0, 64)
     check_status()
+
+
+# --------------------------------------------------------------------------------------------
+# f1, second half: the quantizer hands LayerNorm_i8 its row statistics
+# --------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("path", ["tma", "plain"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("shape", [(32, 32), (96, 160), (64, 4096), (544, 96)])
+def test_quantize_rowstats_bit_exact(shape, dtype, path, monkeypatch):
+    """Codes and scales equal jf_quantize_block's and the oracle's; the per-row, per-block sums of q
+    and q^2 equal the oracle's exactly, on both quantizer kernels and odd block-column counts."""
+    if path == "plain":
+        monkeypatch.setenv("JF_PLAIN_LOADS", "1")
+    rng = np.random.default_rng(zlib.crc32(f"rowstats {shape} {dtype}".encode()))
+    x = S.activation(rng, shape[0], shape[1], max(1, shape[1] // 100), 60.0)
+    x[5, :] = 0.0
+    if dtype == "f32":
+        xd, xh = dev_f32(x), x
+    elif dtype == "bf16":
+        bits = S.to_bf16_bits(x)
+        xd, xh = dev_bf16(bits), O.bf16_bits_to_f32(bits)
+    else:
+        h = S.to_f16(x)
+        xd, xh = torch.from_numpy(h).cuda(), h.astype(np.float32)
+    t, st = jf.quantize_block_rowstats(xd)
+    qr, sr, str_ = O.quantize_block_rowstats(xh)
+    check_status()
+    assert np.array_equal(host(t.q), qr) and np.array_equal(host(t.s), sr)
+    assert np.array_equal(host(st).astype(np.int64), str_)
+
+
+@pytest.mark.parametrize("M,H", [(32, 32), (64, 1024), (96, 4096), (32, 6144), (8192, 4096)])
+def test_layernorm_i8_from_rowstats(M, H):
+    """LayerNorm_i8 with the row statistics from the quantizer against the oracle's LayerNorm_i8 of
+    the same codes, and against the kernel that finds the statistics itself."""
+    rng = np.random.default_rng(zlib.crc32(f"ln rowstats {M} {H}".encode()))
+    x = S.activation(rng, M, H, max(1, H // 100), 50.0)
+    gamma = rng.uniform(0.5, 1.5, H).astype(np.float32)
+    beta = rng.normal(0, 0.2, H).astype(np.float32)
+    X, st = jf.quantize_block_rowstats(dev_f32(x))
+    y = jf.layernorm_i8_rowstats(X, st, dev_f32(gamma), dev_f32(beta), 1e-5)
+    y_ref_gpu = jf.layernorm_i8(X, dev_f32(gamma), dev_f32(beta), 1e-5)
+    check_status()
+    qr, sr = O.quantize_block(x)
+    assert np.array_equal(host(X.q), qr) and np.array_equal(host(X.s), sr)
+    if M <= 96:
+        qo, so, _ = O.layernorm_i8(qr, sr, gamma, beta, 1e-5)
+        assert_requant_close(host(y.q), host(y.s), qo, so, "layernorm_i8 from row stats")
+    else:  # full size: sampled strips against the oracle
+        for r0 in (0, M // 2 - 32, M - 32):
+            qo, so, _ = O.layernorm_i8(qr[r0:r0 + 32], sr[r0 // 32:r0 // 32 + 1], gamma, beta, 1e-5)
+            assert_requant_close(host(y.q)[r0:r0 + 32], host(y.s)[r0 // 32:r0 // 32 + 1], qo, so, "sampled strip")
+    assert_requant_close(host(y.q), host(y.s), host(y_ref_gpu.q), host(y_ref_gpu.s), "from stats vs own pass")
