@@ -58,7 +58,7 @@ __device__ __forceinline__ void store_row_stats(const uint32_t (&w)[2], int* __r
   }
 }
 
-template <typename T>
+template <typename T, bool kStats>
 __global__ void __launch_bounds__(256, 3) quantize_kernel(const T* __restrict__ x, int64_t R, int64_t C,
                                                           int8_t* __restrict__ q, float* __restrict__ s,
                                                           int* __restrict__ stats) {
@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(256, 3) quantize_kernel(const T* __restrict__ 
       for (int g = 0; g < VPG; ++g) Vec<T>::unpack(raw[t + g], *reinterpret_cast<float(*)[EPV]>(v + g * EPV));
       uint32_t w[2];
       quant_pack<8>(v, bq, w);
-      if (stats != nullptr)
+      if constexpr (kStats)
         store_row_stats<EPV, VPG, HALF>(w, stats, bi * 32 + r0 + int64_t(t) * RSTEP, RSTEP, nbc, bj,
                                         active && vc % HALF == 0);
       if (active) {
@@ -149,7 +149,7 @@ __host__ __device__ constexpr int qt_tile_bytes() { return 32 * 64 * int(sizeof(
 template <typename T>
 __host__ __device__ constexpr int qt_smem_bytes() { return QtCfg<T>::kWarps * QtCfg<T>::kDepth * qt_tile_bytes<T>() + 128; }
 
-template <typename T>
+template <typename T, bool kStats>
 __global__ void __launch_bounds__(32 * QtCfg<T>::kWarps, 1) quantize_tma_kernel(const __grid_constant__ CUtensorMap map,
                                                                               int64_t R, int64_t C, int8_t* __restrict__ q,
                                                                               float* __restrict__ s, int* __restrict__ stats,
@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(32 * QtCfg<T>::kWarps, 1) quantize_tma_kernel(
       for (int g = 0; g < VPG; ++g) Vec<T>::unpack(raw[t + g], *reinterpret_cast<float(*)[EPV]>(v + g * EPV));
       uint32_t w[2];
       quant_pack<8>(v, bq, w);
-      if (stats != nullptr)
+      if constexpr (kStats)
         store_row_stats<EPV, VPG, HALF>(w, stats, bi * 32 + r0 + int64_t(t) * RSTEP, RSTEP, nbc, bj,
                                         active && vc % HALF == 0);
       if (active) {
@@ -600,16 +600,17 @@ static bool make_quant_map(CUtensorMap* m, const void* x, int dtype, int64_t R, 
 template <typename T>
 static cudaError_t run_quantize_tma(const CUtensorMap& map, int64_t R, int64_t C, int8_t* q, float* s, int* stats,
                                     unsigned int* status, int sm_count, cudaStream_t st) {
-  static unsigned long long attr_set = 0;  // one bit per device ordinal
-  auto kern = quantize_tma_kernel<T>;
+  static unsigned long long attr_set[2] = {0, 0};  // per variant, one bit per device ordinal
+  auto kern = stats != nullptr ? quantize_tma_kernel<T, true> : quantize_tma_kernel<T, false>;
+  unsigned long long& set = attr_set[stats != nullptr ? 1 : 0];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   const unsigned long long bit = 1ull << (dev & 63);
-  if (!(attr_set & bit)) {
+  if (!(set & bit)) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, qt_smem_bytes<T>());
     if (e != cudaSuccess) return e;
-    attr_set |= bit;
+    set |= bit;
   }
   const int64_t npairs = (R / 32) * ((C / 32 + 1) / 2);
   int64_t grid = (npairs + QtCfg<T>::kWarps - 1) / QtCfg<T>::kWarps;
@@ -629,11 +630,14 @@ cudaError_t launch_quantize(const void* x, int dtype, int64_t R, int64_t C, int8
   // no tensor map for this input (the driver refused it): plain loads
   const int grid = grid_for_blocks((R / 32) * ((C / 32 + 1) / 2), sm_count);  // one warp per block pair
   if (dtype == 0)
-    quantize_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), R, C, q, s, stats);
+    stats != nullptr ? quantize_kernel<float, true><<<grid, 256, 0, st>>>(static_cast<const float*>(x), R, C, q, s, stats)
+                     : quantize_kernel<float, false><<<grid, 256, 0, st>>>(static_cast<const float*>(x), R, C, q, s, stats);
   else if (dtype == 1)
-    quantize_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), R, C, q, s, stats);
+    stats != nullptr ? quantize_kernel<__nv_bfloat16, true><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), R, C, q, s, stats)
+                     : quantize_kernel<__nv_bfloat16, false><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), R, C, q, s, stats);
   else
-    quantize_kernel<__half><<<grid, 256, 0, st>>>(static_cast<const __half*>(x), R, C, q, s, stats);
+    stats != nullptr ? quantize_kernel<__half, true><<<grid, 256, 0, st>>>(static_cast<const __half*>(x), R, C, q, s, stats)
+                     : quantize_kernel<__half, false><<<grid, 256, 0, st>>>(static_cast<const __half*>(x), R, C, q, s, stats);
   return cudaGetLastError();
 }
 
