@@ -109,8 +109,8 @@ __global__ void __launch_bounds__(kLnbThreads, 2) layernorm_i8_bwd_kernel(
     const int8_t* __restrict__ xq, const float* __restrict__ xs, const int8_t* __restrict__ dq,
     const float* __restrict__ ds, int64_t R, int64_t H, const float* __restrict__ gamma, float eps,
     int8_t* __restrict__ qo, float* __restrict__ so, float* __restrict__ part) {
-  __shared__ float4 s_stat[32];  // per row: mean, rstd, mean(g), mean(g xhat)
-  extern __shared__ float s_acc[];  // [2][H] column sums of dy xhat and dy over this CTA's strips
+  __shared__ float4 s_stat[32];  // per row: -mean rstd, rstd, mean(g), mean(g xhat)
+  extern __shared__ __align__(16) float s_acc[];  // [2][H] column sums of dy xhat and dy over this CTA's strips
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t nbc = H >> 5;
   const uint64_t keep = l2_policy_evict_last(), stream = l2_policy_evict_first();
@@ -190,7 +190,10 @@ __global__ void __launch_bounds__(kLnbThreads, 2) layernorm_i8_bwd_kernel(
         const double rstd = 1.0 / sqrt(var + double(eps));
         const double mg = sum_g * inv_h;
         const double mgx = rstd * (sum_gx * inv_h - mean * mg);
-        s_stat[rw] = make_float4(float(mean), float(rstd), float(mg), float(mgx));
+        // -mean rstd as the fp32 product of the rounded mean and rstd, the same value phase 2 formed
+        // per element before: xhat is then exactly 0 where q s equals the mean
+        const float rs = float(rstd);
+        s_stat[rw] = make_float4(-float(mean) * rs, rs, float(mg), float(mgx));
       }
     }
     __syncthreads();
@@ -215,7 +218,7 @@ __global__ void __launch_bounds__(kLnbThreads, 2) layernorm_i8_bwd_kernel(
         i8x4_to_f32(wx[i], fx);
         i8x4_to_f32(wd[i], fd);
         const float4 st = s_stat[rg + 4 * i];
-        const float ax = sx * st.y, bx = -st.x * st.y;  // xhat = q (s rstd) - mean rstd
+        const float ax = sx * st.y, bx = st.x;  // xhat = q (s rstd) - mean rstd
         // dx = rstd (dy gamma - mean(g) - xhat mean(g xhat)), in packed pairs of columns
 #pragma unroll
         for (int j = 0; j < 4; j += 2) {
@@ -238,19 +241,28 @@ __global__ void __launch_bounds__(kLnbThreads, 2) layernorm_i8_bwd_kernel(
       for (int i = 0; i < 8; ++i) st_b32_policy(dst + int64_t(rg + 4 * i) * H + col, o[i], stream);
       if (lane == 0) so[strip * nbc + bj] = bq.s;
       if (part != nullptr) {
+        // column sums over the four row groups (shuffles), then into the CTA's accumulators: the
+        // lane's 4 columns are 16-byte aligned, so one vector load and store each, adds in pairs
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          pgam[j] += __shfl_xor_sync(0xffffffffu, pgam[j], 8);
-          pgam[j] += __shfl_xor_sync(0xffffffffu, pgam[j], 16);
-          pbet[j] += __shfl_xor_sync(0xffffffffu, pbet[j], 8);
-          pbet[j] += __shfl_xor_sync(0xffffffffu, pbet[j], 16);
+        for (int o = 8; o <= 16; o <<= 1) {
+#pragma unroll
+          for (int j = 0; j < 4; j += 2) {
+            add_x2(pgam[j], pgam[j + 1], __shfl_xor_sync(0xffffffffu, pgam[j], o),
+                   __shfl_xor_sync(0xffffffffu, pgam[j + 1], o), pgam[j], pgam[j + 1]);
+            add_x2(pbet[j], pbet[j + 1], __shfl_xor_sync(0xffffffffu, pbet[j], o),
+                   __shfl_xor_sync(0xffffffffu, pbet[j + 1], o), pbet[j], pbet[j + 1]);
+          }
         }
         if (rg == 0) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            s_acc[col + j] += pgam[j];
-            s_acc[H + col + j] += pbet[j];
-          }
+          float4* ag = reinterpret_cast<float4*>(s_acc + col);
+          float4* ab = reinterpret_cast<float4*>(s_acc + H + col);
+          float4 g = *ag, b = *ab;
+          add_x2(g.x, g.y, pgam[0], pgam[1], g.x, g.y);
+          add_x2(g.z, g.w, pgam[2], pgam[3], g.z, g.w);
+          add_x2(b.x, b.y, pbet[0], pbet[1], b.x, b.y);
+          add_x2(b.z, b.w, pbet[2], pbet[3], b.z, b.w);
+          *ag = g;
+          *ab = b;
         }
       }
     }
