@@ -28,7 +28,10 @@
  * Execution: every call validates its arguments on the host, returns an error code without
  * enqueuing anything if they are invalid, otherwise enqueues its kernel(s) on `stream` (a
  * cudaStream_t passed as void*; NULL = the legacy default stream) and returns without waiting.
- * The library never allocates, frees or retains device memory. Outputs must not overlap inputs.
+ * The library allocates, frees and retains no device memory of its own per call: every buffer is
+ * the caller's. The one exception is a 16 MiB static scratch array that the library's module holds
+ * on each device where it is loaded, used only by jf_layernorm_i8_bwd_noalloc. Resetting a device
+ * (cudaDeviceReset) while the library is loaded is not supported. Outputs must not overlap inputs.
  * Inputs must be finite. Kernel-side failures (a bounded wait that timed out) are reported by
  * jf_device_status(). Calls are thread-safe; calls on different streams may run concurrently.
  * There is no CPU fallback: on a machine without an sm_100 GPU every compute call returns
@@ -94,8 +97,9 @@ typedef enum { JF_GRAN_BLOCK = 0, JF_GRAN_TOKEN = 1, JF_GRAN_CHANNEL = 2, JF_GRA
  * Codes and scales are bit-exact with the rule above (bf16/fp16 are widened exactly first).
  * The kernel stages x through shared memory with TMA tile loads and waits on them with bounded
  * waits: if one runs out, the kernel gives up and jf_device_status reports JF_ERR_TIMEOUT. With
- * JF_PLAIN_LOADS=1 in the environment (read on every call) a kernel with plain loads runs instead
- * (the path for inputs the driver cannot describe with a tensor map); its results are identical.
+ * JF_PLAIN_LOADS=1 in the environment when the library is loaded (read once, at load time) a kernel
+ * with plain loads runs instead (the path for inputs the driver cannot describe with a tensor map);
+ * its results are identical.
  */
 JF_API int jf_quantize_block(const void* x, jf_dtype dt, int64_t rows, int64_t cols, int8_t* q, float* s,
                       void* stream);
@@ -222,13 +226,14 @@ JF_API int64_t jf_layernorm_i8_bwd_workspace_bytes(int64_t rows, int64_t cols);
 
 /*
  * Allocation-free variant of jf_layernorm_i8_bwd (no counterpart on the pages: an engineering entry
- * point for callers that cannot provide a workspace). Same arguments, results and errors, but the
- * per-CTA column sums go to a 16 MiB scratch array that the library holds in device memory for
- * its whole lifetime, so neither the caller nor the library allocates anything per call. Shapes
- * whose workspace (jf_layernorm_i8_bwd_workspace_bytes) exceeds 16 MiB are rejected with
- * JF_ERR_WORKSPACE before anything is enqueued. The scratch is shared by every call on a device:
- * calls of this function that ask for dgamma or dbeta must not run concurrently with each other
- * (issue them on one stream). Without dgamma and dbeta it is jf_layernorm_i8_bwd with no workspace.
+ * point for callers that cannot provide a workspace). Same arguments, results and errors, checked in
+ * the same order, but the per-CTA column sums go to a 16 MiB scratch array that the library holds in
+ * device memory for its whole lifetime, so neither the caller nor the library allocates anything per
+ * call. After every other argument check has passed, shapes whose workspace
+ * (jf_layernorm_i8_bwd_workspace_bytes) exceeds 16 MiB are rejected with JF_ERR_WORKSPACE before
+ * anything is enqueued. The scratch is shared by every call on a device: calls of this function that
+ * ask for dgamma or dbeta must not run concurrently with each other (issue them on one stream).
+ * Without dgamma and dbeta it is jf_layernorm_i8_bwd with no workspace.
  */
 JF_API int jf_layernorm_i8_bwd_noalloc(jf_cqtensor X, jf_cqtensor dY, const float* gamma, float eps,
                                        jf_qtensor dX, float* dgamma, float* dbeta, void* stream);
@@ -254,10 +259,10 @@ JF_API int jf_dequantize_granular(const int8_t* q, const float* s, int64_t rows,
 
 /*
  * f3. The error of a quantization (the summary's accuracy metric behind the ablation): writes
- *     sums[0] = sum over elements of (x - q s)^2 and sums[1] = sum of x^2, in fp64, to the device
- *     array `sums` (2 doubles, 8-byte aligned); x, q and s as above, all exact in fp64, so only the
- *     order of the fp64 additions (unspecified) affects the result. The mean squared error is
- *     sums[0] / (rows * cols).
+ *     sums[0] = sum over elements of (x - q s)^2, sums[1] = sum of x^2 and
+ *     sums[2] = sums[0] / (rows * cols), the mean squared error, in fp64 to the device array `sums`
+ *     (3 doubles, 8-byte aligned); x, q and s as above, all exact in fp64, so only the order of the
+ *     fp64 additions (unspecified) affects the sums. An empty tensor gives three zeros.
  */
 JF_API int jf_quantization_error(const void* x, jf_dtype dt, const int8_t* q, const float* s, int64_t rows,
                                  int64_t cols, jf_granularity g, double* sums, void* stream);

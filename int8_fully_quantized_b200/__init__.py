@@ -294,9 +294,9 @@ def quantize_granular(x: torch.Tensor, granularity: str, stream=None):
 def quantization_mse(x: torch.Tensor, granularity: str, stream=None) -> float:
     """Mean squared error of quantize -> dequantize at one granularity, computed on the GPU."""
     q, s = quantize_granular(x, granularity, stream)
-    sums = torch.empty(2, dtype=torch.float64, device=x.device)
+    sums = torch.empty(3, dtype=torch.float64, device=x.device)
     jf_quantization_error(x, q, s, GRANULARITY[granularity], sums, stream)
-    return float(sums[0].item()) / x.numel()
+    return float(sums[2].item())
 
 
 def jf_mx_quantize(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, stream=None) -> None:

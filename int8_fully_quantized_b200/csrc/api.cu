@@ -1,6 +1,7 @@
 // C ABI of the library: argument validation, then the kernel launch (see include/jetfire.h).
 #include <cstdint>
 #include <cstdlib>
+#include <mutex>
 #include <cuda_runtime.h>
 
 #include "jetfire.h"
@@ -19,8 +20,12 @@ struct DevInfo {
   unsigned int* status = nullptr;  // device address of jf::g_status on this device
 };
 
-// Per-device SM count and capability check (cached per device ordinal).
+// Per-device SM count and capability check (cached per device ordinal; the first call on a device
+// fills its entry under a lock, so concurrent first calls from several threads are safe). The
+// cached status-word address belongs to the device's primary context: resetting the device
+// (cudaDeviceReset) while the library is loaded is not supported.
 DevInfo device_info() {
+  static std::mutex mu;
   static DevInfo cache[64];
   static bool probed[64] = {false};
   int dev = -1;
@@ -28,6 +33,7 @@ DevInfo device_info() {
     cudaGetLastError();
     return DevInfo{};
   }
+  std::lock_guard<std::mutex> lock(mu);
   if (!probed[dev]) {
     DevInfo d;
     int major = 0, sms = 0;
@@ -63,12 +69,14 @@ inline bool overlap(const void* a, int64_t na, const void* b, int64_t nb) {
 inline int64_t elem_size(jf_dtype dt) { return dt == JF_F32 ? 4 : 2; }
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? JF_OK : JF_ERR_CUDA; }
 
-// JF_PLAIN_LOADS=1 in the environment (read on every call) selects the quantizer's plain-load kernel,
-// which otherwise serves only inputs the driver will not describe with a TMA tensor map.
-inline bool plain_loads_forced() {
+// JF_PLAIN_LOADS=1 in the environment when the library is loaded selects the quantizer's plain-load
+// kernel, which otherwise serves only inputs the driver will not describe with a TMA tensor map. The
+// variable is read once, at load time, so no call reads the environment.
+const bool g_plain_loads = [] {
   const char* v = std::getenv("JF_PLAIN_LOADS");
   return v != nullptr && v[0] == '1';
-}
+}();
+inline bool plain_loads_forced() { return g_plain_loads; }
 
 int check_cq(const jf_cqtensor& t) {
   if (!dims_ok(t.rows, t.cols)) return JF_ERR_SHAPE;
@@ -310,8 +318,14 @@ int64_t jf_layernorm_i8_bwd_workspace_bytes(int64_t rows, int64_t cols) {
   return jf::ln_bwd_ctas(rows) * 2 * cols * 4;
 }
 
-int jf_layernorm_i8_bwd(jf_cqtensor X, jf_cqtensor dY, const float* gamma, float eps, jf_qtensor dX, float* dgamma,
-                        float* dbeta, void* workspace, int64_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+// Every check of the LayerNorm backward that does not involve the workspace, in the order both
+// entry points apply them: tensors, shapes, NULL gamma, alignment, then overlaps among the
+// inputs and outputs (the workspace is checked by the caller of this function).
+int ln_bwd_validate(const jf_cqtensor& X, const jf_cqtensor& dY, const float* gamma, const jf_qtensor& dX,
+                    const float* dgamma, const float* dbeta) {
   int st;
   if ((st = check_cq(X)) != JF_OK) return st;
   if ((st = check_cq(dY)) != JF_OK) return st;
@@ -321,43 +335,64 @@ int jf_layernorm_i8_bwd(jf_cqtensor X, jf_cqtensor dY, const float* gamma, float
   if (X.rows == 0 || X.cols == 0) return JF_OK;
   if (gamma == nullptr) return JF_ERR_NULL;
   if (!aligned(gamma, 16) || !aligned(dgamma, 4) || !aligned(dbeta, 4)) return JF_ERR_ALIGN;
-  const bool want_param_grads = dgamma != nullptr || dbeta != nullptr;
-  if (want_param_grads &&
-      (workspace == nullptr || !aligned(workspace, 16) ||
-       workspace_bytes < jf_layernorm_i8_bwd_workspace_bytes(X.rows, X.cols)))
-    return JF_ERR_WORKSPACE;
   const int64_t nq = qbytes(X), ns = sbytes(X.rows, X.cols), H = X.cols;
-  const int64_t nw = want_param_grads ? jf_layernorm_i8_bwd_workspace_bytes(X.rows, X.cols) : 0;
   const void* ins[5] = {X.q, X.s, dY.q, dY.s, gamma};
   const int64_t in_n[5] = {nq, ns, nq, ns, H * 4};
-  const void* outs[5] = {dX.q, dX.s, dgamma, dbeta, want_param_grads ? workspace : nullptr};
-  const int64_t out_n[5] = {nq, ns, H * 4, H * 4, nw};
-  for (int o = 0; o < 5; ++o) {
+  const void* outs[4] = {dX.q, dX.s, dgamma, dbeta};
+  const int64_t out_n[4] = {nq, ns, H * 4, H * 4};
+  for (int o = 0; o < 4; ++o) {
     for (int i = 0; i < 5; ++i)
       if (overlap(outs[o], out_n[o], ins[i], in_n[i])) return JF_ERR_ALIAS;
-    for (int o2 = o + 1; o2 < 5; ++o2)
+    for (int o2 = o + 1; o2 < 4; ++o2)
       if (overlap(outs[o], out_n[o], outs[o2], out_n[o2])) return JF_ERR_ALIAS;
   }
+  return JF_OK;
+}
+
+// The launch shared by both entry points, after validation. `part` is the column-sum workspace
+// (NULL when neither dgamma nor dbeta is wanted).
+int ln_bwd_launch(const jf_cqtensor& X, const jf_cqtensor& dY, const float* gamma, float eps, const jf_qtensor& dX,
+                  float* dgamma, float* dbeta, float* part, void* stream) {
   const DevInfo d = device_info();
   if (!d.ok) return JF_ERR_DEVICE;
-  return cuda_status(jf::launch_layernorm_i8_bwd(X.q, X.s, dY.q, dY.s, X.rows, X.cols, gamma, eps, dX.q, dX.s,
-                                                 want_param_grads ? static_cast<float*>(workspace) : nullptr,
+  return cuda_status(jf::launch_layernorm_i8_bwd(X.q, X.s, dY.q, dY.s, X.rows, X.cols, gamma, eps, dX.q, dX.s, part,
                                                  dgamma, dbeta, static_cast<cudaStream_t>(stream)));
+}
+}  // namespace
+
+extern "C" {
+
+int jf_layernorm_i8_bwd(jf_cqtensor X, jf_cqtensor dY, const float* gamma, float eps, jf_qtensor dX, float* dgamma,
+                        float* dbeta, void* workspace, int64_t workspace_bytes, void* stream) {
+  int st;
+  if ((st = ln_bwd_validate(X, dY, gamma, dX, dgamma, dbeta)) != JF_OK) return st;
+  if (X.rows == 0 || X.cols == 0) return JF_OK;
+  const bool want_param_grads = dgamma != nullptr || dbeta != nullptr;
+  if (!want_param_grads) return ln_bwd_launch(X, dY, gamma, eps, dX, nullptr, nullptr, nullptr, stream);
+  const int64_t nw = jf_layernorm_i8_bwd_workspace_bytes(X.rows, X.cols);
+  if (workspace == nullptr || !aligned(workspace, 16) || workspace_bytes < nw) return JF_ERR_WORKSPACE;
+  const int64_t nq = qbytes(X), ns = sbytes(X.rows, X.cols), H = X.cols;
+  const void* others[7] = {X.q, X.s, dY.q, dY.s, gamma, dX.q, dX.s};
+  const int64_t other_n[7] = {nq, ns, nq, ns, H * 4, nq, ns};
+  for (int i = 0; i < 7; ++i)
+    if (overlap(workspace, nw, others[i], other_n[i])) return JF_ERR_ALIAS;
+  if (overlap(workspace, nw, dgamma, H * 4) || overlap(workspace, nw, dbeta, H * 4)) return JF_ERR_ALIAS;
+  return ln_bwd_launch(X, dY, gamma, eps, dX, dgamma, dbeta, static_cast<float*>(workspace), stream);
 }
 
 int jf_layernorm_i8_bwd_noalloc(jf_cqtensor X, jf_cqtensor dY, const float* gamma, float eps, jf_qtensor dX,
                                 float* dgamma, float* dbeta, void* stream) {
-  if (dgamma == nullptr && dbeta == nullptr)
-    return jf_layernorm_i8_bwd(X, dY, gamma, eps, dX, nullptr, nullptr, nullptr, 0, stream);
-  const int64_t need = jf_layernorm_i8_bwd_workspace_bytes(X.rows, X.cols);
-  if (need < 0) return JF_ERR_SHAPE;
-  if (need > jf::kLnBwdScratchBytes) return JF_ERR_WORKSPACE;  // larger than the static scratch
-  if (X.rows == 0 || X.cols == 0) return jf_layernorm_i8_bwd(X, dY, gamma, eps, dX, dgamma, dbeta, nullptr, 0, stream);
+  // the same argument checks, in the same order, as jf_layernorm_i8_bwd; only then the scratch size
+  int st;
+  if ((st = ln_bwd_validate(X, dY, gamma, dX, dgamma, dbeta)) != JF_OK) return st;
+  if (X.rows == 0 || X.cols == 0) return JF_OK;
+  if (dgamma == nullptr && dbeta == nullptr) return ln_bwd_launch(X, dY, gamma, eps, dX, nullptr, nullptr, nullptr, stream);
+  if (jf_layernorm_i8_bwd_workspace_bytes(X.rows, X.cols) > jf::kLnBwdScratchBytes) return JF_ERR_WORKSPACE;
   const DevInfo d = device_info();
   if (!d.ok) return JF_ERR_DEVICE;
   float* scratch = jf::ln_bwd_static_scratch();
   if (scratch == nullptr) return JF_ERR_CUDA;
-  return jf_layernorm_i8_bwd(X, dY, gamma, eps, dX, dgamma, dbeta, scratch, jf::kLnBwdScratchBytes, stream);
+  return ln_bwd_launch(X, dY, gamma, eps, dX, dgamma, dbeta, scratch, stream);
 }
 
 int64_t jf_granular_scale_count(int64_t rows, int64_t cols, jf_granularity g) {
@@ -419,12 +454,12 @@ int jf_quantization_error(const void* x, jf_dtype dt, const int8_t* q, const flo
   if (rows != 0 && cols != 0) {
     if (x == nullptr || q == nullptr || s == nullptr) return JF_ERR_NULL;
     if (!aligned(x, 16) || !aligned(q, 16) || !aligned(s, 4)) return JF_ERR_ALIGN;
-    if (overlap(sums, 16, x, nx) || overlap(sums, 16, q, rows * cols) || overlap(sums, 16, s, ns)) return JF_ERR_ALIAS;
+    if (overlap(sums, 24, x, nx) || overlap(sums, 24, q, rows * cols) || overlap(sums, 24, s, ns)) return JF_ERR_ALIAS;
   }
   const DevInfo d = device_info();
   if (!d.ok) return JF_ERR_DEVICE;
   if (rows == 0 || cols == 0)
-    return cuda_status(cudaMemsetAsync(sums, 0, 2 * sizeof(double), static_cast<cudaStream_t>(stream)));
+    return cuda_status(cudaMemsetAsync(sums, 0, 3 * sizeof(double), static_cast<cudaStream_t>(stream)));
   return cuda_status(jf::launch_quant_error(x, int(dt), q, s, rows, cols, int(g), sums, d.sm_count,
                                             static_cast<cudaStream_t>(stream)));
 }

@@ -305,8 +305,11 @@ __global__ void __launch_bounds__(256) ln_bwd_reduce_kernel(const float* __restr
 
 // ---------------------------------------------------------------------------------------------
 // Static scratch of the allocation-free LayerNorm backward: the per-CTA column sums live in this
-// file-scope device array instead of a caller workspace. Its device address is looked up once per
-// device and cached.
+// file-scope device array instead of a caller workspace. In host code the array's name only stands
+// for the symbol, so its device address is looked up (cudaGetSymbolAddress) once per device, with
+// that device current, and cached; the cache belongs to the device's primary context, so resetting
+// the device (cudaDeviceReset) while the library is loaded is not supported. A failed lookup clears
+// the CUDA error it raised, so that it does not surface in a later call.
 // ---------------------------------------------------------------------------------------------
 static __device__ __align__(256) float g_ln_bwd_scratch[kLnBwdScratchBytes / sizeof(float)];
 
@@ -314,11 +317,17 @@ float* ln_bwd_static_scratch() {
   static std::mutex mu;
   static float* addr[64] = {};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return nullptr;
+  }
   std::lock_guard<std::mutex> lock(mu);
   if (addr[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_ln_bwd_scratch) != cudaSuccess) return nullptr;
+    if (cudaGetSymbolAddress(&p, g_ln_bwd_scratch) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
     addr[dev] = static_cast<float*>(p);
   }
   return addr[dev];

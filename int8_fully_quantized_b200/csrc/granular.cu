@@ -222,6 +222,10 @@ __global__ void __launch_bounds__(kGranThreads) quant_error_kernel(const T* __re
   }
 }
 
+// The mean squared error from the two sums: sums[2] = sums[0] / n (one IEEE fp64 division), after
+// every CTA of quant_error_kernel has added its part.
+__global__ void quant_error_mse_kernel(double* __restrict__ sums, double n) { sums[2] = sums[0] / n; }
+
 // ---------------------------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------------------------
@@ -289,7 +293,7 @@ template <typename T>
 static cudaError_t quant_error_t(const T* x, const int8_t* q, const float* s, int64_t R, int64_t C, int g,
                                  double* sums, int sm_count, cudaStream_t st) {
   const int grid = grid_for(R * (C / Vec<T>::kElems), kGranThreads, sm_count, 4);
-  cudaError_t e = cudaMemsetAsync(sums, 0, 2 * sizeof(double), st);
+  cudaError_t e = cudaMemsetAsync(sums, 0, 3 * sizeof(double), st);
   if (e != cudaSuccess) return e;
   switch (g) {
     case kGranBlock: quant_error_kernel<T, kGranBlock><<<grid, kGranThreads, 0, st>>>(x, q, s, R, C, sums); break;
@@ -297,6 +301,9 @@ static cudaError_t quant_error_t(const T* x, const int8_t* q, const float* s, in
     case kGranChannel: quant_error_kernel<T, kGranChannel><<<grid, kGranThreads, 0, st>>>(x, q, s, R, C, sums); break;
     default: quant_error_kernel<T, kGranTensor><<<grid, kGranThreads, 0, st>>>(x, q, s, R, C, sums); break;
   }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  quant_error_mse_kernel<<<1, 1, 0, st>>>(sums, double(R) * double(C));
   return cudaGetLastError();
 }
 

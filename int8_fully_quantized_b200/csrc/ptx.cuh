@@ -7,9 +7,8 @@
 
 namespace jf {
 
-// Bits of the library's device status word (read and cleared by jf_device_status).
+// Bit of the library's device status word (read and cleared by jf_device_status).
 constexpr unsigned int kStatusTimeout = 1u;   // a bounded wait ran out
-constexpr unsigned int kStatusBounds = 2u;    // a kernel refused an out-of-range access
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long kWatchdogNs = 4000000000ull;

@@ -15,7 +15,7 @@ computation with per-block scales. The "Fp8 vs int8" page gives the signed INT8 
 dequantization x = FP(q) * s.
 
 The pages state no formula for the scale, no rounding mode and no accumulation order. The
-readings taken here (each listed in the design doc):
+readings taken here:
 
 * square 32x32 blocks, scale s = absmax(block) / 127 in fp32 (IEEE division), no zero point;
 * q = clamp(rint(x / s), -127, 127): fp32 IEEE division, then round-half-to-even; -128 is never

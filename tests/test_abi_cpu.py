@@ -106,9 +106,21 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert lib.jf_layernorm_i8_bwd(Xc, dYc, None, f, dXq, dg, db, ws, need, None) == -1
     assert lib.jf_layernorm_i8_bwd(Xc, dYc, g, f, dXq, dg, vp((1 << 33) + 8), ws, need, None) == -5
     assert lib.jf_layernorm_i8_bwd(Xc, dYc, g, f, dXq, dg, db, vp((1 << 34) + 16), need, None) == -5
-    # the allocation-free backward refuses shapes whose column sums exceed its 16 MiB static scratch
-    big = jf._CQ(1 << 20, 1 << 22, 32768, 8192)
-    assert lib.jf_layernorm_i8_bwd_noalloc(big, big, g, f, jf._Q(1 << 28, 1 << 30, 32768, 8192), dg, db, None) == -9
+    # the allocation-free backward refuses shapes whose column sums exceed its 16 MiB static scratch,
+    # but only after the argument checks of the workspace version (same errors, same order)
+    R, H = 9472, 7104                      # 296 CTAs x 2 x 7104 x 4 bytes = 16.04 MiB, just above the limit
+    assert lib.jf_layernorm_i8_bwd_workspace_bytes(R, H) == 296 * 2 * H * 4 > 16 << 20
+    Xb, dYb = jf._CQ(1 << 36, 1 << 37, R, H), jf._CQ(1 << 38, 1 << 39, R, H)
+    dXb = jf._Q(1 << 40, 1 << 41, R, H)
+    gb, dgb, dbb = vp(1 << 42), vp(1 << 43), vp(1 << 44)
+    assert lib.jf_layernorm_i8_bwd_noalloc(Xb, dYb, gb, f, dXb, dgb, dbb, None) == -9
+    assert lib.jf_layernorm_i8_bwd_noalloc(Xb, dYb, gb, f, jf._Q(None, 1 << 41, R, H), dgb, dbb, None) == -1
+    assert lib.jf_layernorm_i8_bwd_noalloc(Xb, jf._CQ(1 << 38, 1 << 39, R, H - 32), gb, f, dXb, dgb, dbb, None) == -2
+    assert lib.jf_layernorm_i8_bwd_noalloc(Xb, dYb, vp((1 << 42) + 4), f, dXb, dgb, dbb, None) == -3
+    assert lib.jf_layernorm_i8_bwd_noalloc(Xb, dYb, None, f, dXb, dgb, dbb, None) == -1
+    assert lib.jf_layernorm_i8_bwd_noalloc(Xb, dYb, gb, f, jf._Q(1 << 36, 1 << 41, R, H), dgb, dbb, None) == -5
+    # without dgamma and dbeta there is no scratch, so no size limit other than H <= 24576
+    assert lib.jf_layernorm_i8_bwd_noalloc(Xb, dYb, gb, f, jf._Q(None, 1 << 41, R, H), None, None, None) == -1
     # granularity variants: unknown granularity, scale counts
     assert lib.jf_quantize_granular(fake, 1, 32, 64, 7, fake, fake, None) == -10
     assert [lib.jf_granular_scale_count(64, 96, g) for g in range(4)] == [6, 64, 96, 1]
@@ -136,5 +148,12 @@ def test_compute_without_gpu_fails_loudly(lib):
     # valid arguments, but no sm_100 device is current: the call must refuse, never fall back
     st = lib.jf_quantize_block(vp(1 << 20), 1, 32, 32, vp(1 << 24), vp(1 << 26), None)
     assert st == -8
+    # the allocation-free LayerNorm backward at the largest shape its static scratch takes
+    # (296 x 2 x 7072 x 4 bytes = 15.97 MiB) passes every host check and stops only at the device
+    R, H = 9472, 7072
+    assert lib.jf_layernorm_i8_bwd_workspace_bytes(R, H) <= 16 << 20
+    assert lib.jf_layernorm_i8_bwd_noalloc(jf._CQ(1 << 36, 1 << 37, R, H), jf._CQ(1 << 38, 1 << 39, R, H),
+                                           vp(1 << 42), ctypes.c_float(1e-5), jf._Q(1 << 40, 1 << 41, R, H),
+                                           vp(1 << 43), vp(1 << 44), None) == -8
     with pytest.raises(jf.JetfireError):
         jf._check(st, "jf_quantize_block")

@@ -62,9 +62,10 @@ def test_quantization_error_sums(g):
     x32 = S.activation(rng, rows, cols, 10, 30.0)
     xd, xh = _device_input(x32, "bf16")
     q, s = jf.quantize_granular(xd, g)
-    sums = torch.empty(2, dtype=torch.float64, device="cuda")
+    sums = torch.empty(3, dtype=torch.float64, device="cuda")
     jf.jf_quantization_error(xd, q, s, jf.GRANULARITY[g], sums)
     got = host(sums)
+    assert got[2] == got[0] / x32.size     # the MSE is the first sum over the element count
     br, bc = _block_shape(g, rows, cols)
     qr, sr = O.quantize(xh, br, bc)
     xr = qr.astype(np.float64) * O.block_scale_grid(sr, br, bc).astype(np.float64)
@@ -83,4 +84,16 @@ def test_ablation_direction_on_the_gpu():
     xd = dev_bf16(S.to_bf16_bits(d["X"]))
     mse = {g: jf.quantization_mse(xd, g) for g in ["block", "token", "channel", "tensor"]}
     assert mse["block"] < mse["token"] <= mse["tensor"]
+    check_status()
+
+
+@pytest.mark.parametrize("g", ["block"] + GRAN)
+def test_quantization_mse_hand_worked_on_the_gpu(g):
+    """The hand-worked quarter-offset input (every non-absmax element coded with an error of exactly
+    s/4): the GPU's MSE must equal (1 - n_max / n) s^2 / 16 exactly, since every term and partial sum
+    is a multiple of 2^-10 well inside fp64."""
+    from test_oracle_pins import quarter_offset_input
+    x, expected = quarter_offset_input(g)
+    xd = torch.from_numpy(x).cuda()
+    assert jf.quantization_mse(xd, g) == expected
     check_status()

@@ -138,6 +138,40 @@ def test_granularity_mse_direction():
     assert mb < mt <= mT * 1.0000001
 
 
+def quarter_offset_input(granularity, rows=64, cols=64, exp=-3, seed=9):
+    """An fp32 [rows, cols] tensor whose quantization error is known by hand at one granularity.
+
+    Every group of the granularity holds one element of magnitude exactly 127 s (s = 2**exp), so
+    its scale is exactly s and that element is coded without error; every other element is
+    (n + 1/4) s with an integer |n| <= 100, which the quantizer codes as n, an error of exactly s/4.
+    The mean squared error is therefore (1 - n_max / (rows*cols)) * s^2 / 16, with n_max the number
+    of +-127 s elements. Returns (x, expected_mse)."""
+    rng = np.random.default_rng(seed)
+    s = np.float32(2.0 ** exp)
+    x = (rng.integers(-100, 101, size=(rows, cols)).astype(np.float32) + np.float32(0.25)) * s
+    br, bc = {"block": (32, 32), "token": (1, cols), "channel": (rows, 1), "tensor": (rows, cols)}[granularity]
+    for I in range(rows // br):
+        for J in range(cols // bc):
+            r, c = I * br + int(rng.integers(0, br)), J * bc + int(rng.integers(0, bc))
+            x[r, c] = np.float32(127.0) * s * np.float32(1 if rng.integers(0, 2) else -1)
+    n_max = int(np.count_nonzero(np.abs(x) == np.float32(127.0) * s))
+    return x.astype(np.float32), (1.0 - n_max / x.size) * float(s) ** 2 / 16.0
+
+
+@pytest.mark.parametrize("granularity", ["block", "token", "channel", "tensor"])
+def test_quantization_mse_hand_worked(granularity):
+    """Hand-worked value of the quantization MSE: quarter-offset codes give an error of exactly s/4
+    per element (s^2/16 squared) except at each group's absmax, which is exact. A sum instead of a
+    mean, an absolute instead of a squared error, or a scale taken at the wrong granularity gives
+    another number."""
+    x, expected = quarter_offset_input(granularity)
+    assert O.quantization_mse(x, granularity) == expected
+    # built for one scale per tensor, the input has blocks without a 127 s element: their scales are
+    # not s, so at the 32x32 granularity the error is another number
+    if granularity == "tensor":
+        assert O.quantization_mse(x, "block") != expected
+
+
 # ---------------------------------------------------------------------------------------------
 # dtype conversions and dequantize
 # ---------------------------------------------------------------------------------------------
