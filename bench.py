@@ -1,21 +1,27 @@
 #!/usr/bin/env python
 """Benchmark of the per-block INT8 data-flow hot path on B200.
 
-One step = one pass of every operator of the path over one batch of the GPT2-medium MLP linear
-workload (tokens M = 4096, hidden K = 1024, N = 4096; X ~ N(0,1) with 1% of the channels x30,
-W ~ N(0, 0.02), dY ~ N(0, 1e-3), bf16 on entry):
+One step = one training pass (forward and backward) of the hidden-4096 transformer MLP layer on INT8
+blocks, M = 8192 tokens, hidden H = 4096, inner F = 16384 (the hidden-4096 layer of the Jetfire
+summary's "Key results" and "Measured effects" table): X ~ N(0,1) with 4 outlier channels x50, W1 and
+W2 ~ N(0, 0.02), the upstream gradient dY ~ N(0, 1e-3), all bf16 on entry:
 
-    quantize X -> LayerNorm_i8 -> quantize W -> linear fwd (Y = X W^T) -> GELU_i8
-    quantize dY -> dgrad (dX = dY W) -> wgrad (dW = dY^T X) -> dequantize dX to bf16
+    forward:  quantize X -> LayerNorm_i8 -> fc1 (Y1 = Xn W1^T) -> GELU_i8 -> fc2 (Y2 = G W2^T)
+              (quantize W1, W2 beside them)
+    backward: quantize dY -> fc2 dgrad (dG = dY W2) and wgrad (dW2 = dY^T G) -> GELU_i8 backward
+              -> fc1 dgrad (dXn = dY1 W1) and wgrad (dW1 = dY1^T Xn) -> LayerNorm_i8 backward
+              (dX, dgamma, dbeta) -> dequantize dX to bf16
 
-Inputs are resident in HBM when the timed region starts; L2 is flushed between steps (a 256 MiB
-write outside the timed events). ``value`` is the whole-step throughput in TOPS counted on the
-three GEMMs (3 x 2MNK int8 ops per step and rank) over the step time, summed over ranks.
-``--gpus N`` (under torchrun) runs N data-parallel ranks, each with its own M = 4096 tokens; the
-fp32 weight-gradient partials are summed with NCCL and re-quantized (weak scaling).
+Every operator reads and writes INT8 blocks with per-block scales; six block-scaled INT8 GEMMs of
+2 * 8192 * 4096 * 16384 int8 ops each. Inputs are resident in HBM when the timed region starts; L2
+is flushed between steps (a 256 MiB write outside the timed events). ``value`` is the whole-step
+throughput in TOPS counted on the six GEMMs over the step time, summed over ranks. ``--gpus N``
+(under torchrun) runs N data-parallel ranks, each with its own 8192 tokens; the fp32 weight-gradient
+partials are summed with NCCL all-reduces that overlap the rest of the backward, then re-quantized
+(weak scaling).
 
 ``--impl reference`` times the CPU oracle (the method written out plainly in numpy) on a bounded
-token sample of the same workload, on rank 0 only.
+sample of the same workload, on rank 0 only.
 """
 from __future__ import annotations
 
@@ -34,23 +40,30 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "per-block INT8 GEMM TOPS (% INT8 peak); quantize/GELU/LN GB/s (% HBM)"
-WORKLOAD = "gpt2m_fc1"
+WORKLOAD_NAME = ("hidden-4096 MLP layer on INT8 blocks, forward and backward: LayerNorm_i8 -> fc1 4096->16384 -> "
+                 "GELU_i8 -> fc2 16384->4096, six block-scaled INT8 GEMMs (fwd, dgrad, wgrad of fc1 and fc2), "
+                 "quantize, GELU_i8 and LayerNorm_i8 backward, dequantize (per rank)")
 NOMINAL_I8_OVER_BF16 = 2.0       # dense int8 (4.5 POPS) / dense bf16 (2.25 PFLOP/s), nominal B200
+NOMINAL_I8_TOPS = 4500.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+ALU_LANES_PER_CLK_PER_SM = 128   # 4 warp schedulers x 32 lanes, one issue per scheduler per clock
+B200_SMS = 148
 
 
 def parse_args():
     p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=50)
-    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     p.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    p.add_argument("--no-sweep", action="store_true", help="skip the memory-bound sweep in the main line")
     p.add_argument("--eager", action="store_true", help="time eager launches instead of the step's CUDA graph")
     p.add_argument("--configs", action="store_true",
                    help="time the single-linear, hidden-4096 GEMM and hidden-4096 MLP-block workloads (one JSON line)")
-    p.add_argument("--cpu-sample-tokens", type=int, default=1024)
+    p.add_argument("--cpu-sample-blocks", type=int, default=16,
+                   help="oracle sample: this many x this many output blocks of each GEMM")
     p.add_argument("--sweep", action="store_true",
                    help="time the memory-bound kernels on the M x 4096 sweep instead of the step")
     p.add_argument("--sweep-m", type=int, nargs="*", default=[1024, 8192, 65536])
@@ -58,10 +71,6 @@ def parse_args():
                                                       "gelu_i8_bwd", "layernorm_i8_bwd", "fused_fc1",
                                                       "granularity_mse", "mxfp8_fc1"])
     return p.parse_args()
-
-
-ALU_LANES_PER_CLK_PER_SM = 128   # 4 warp schedulers x 32 lanes, one issue per scheduler per clock
-B200_SMS = 148
 
 
 def load_peaks():
@@ -149,87 +158,184 @@ class ClockSampler:
 # --------------------------------------------------------------------------------------------
 # host inputs
 # --------------------------------------------------------------------------------------------
-def host_inputs(M, K, N, seed_tokens, seed_weight):
+def layer_dims():
     from inputs import synthetic as S
-    w = S.WORKLOADS[WORKLOAD]
+    w = S.WORKLOADS["h4096_fc1"]
+    return w["M"], w["K"], w["N"]          # tokens M, hidden H, inner F
+
+
+def host_inputs(seed_tokens, seed_weight, dims=None):
+    """bf16 bit patterns of X [M, H], dY [M, H], W1 [F, H], W2 [H, F]; fp32 gamma, beta [H]
+    (dims = (M, H, F), the layer's by default)."""
+    from inputs import synthetic as S
+    M, H, F = dims or layer_dims()
+    n_out, fac = S.WORKLOADS["h4096_fc1"]["x_outliers"]
     rng = np.random.default_rng(seed_tokens)
+    x = S.activation(rng, M, H, n_out, fac)
+    dy = S.grad(rng, M, H)
+    rw = np.random.default_rng(seed_weight)
+    w1 = S.weight(rw, F, H)
+    w2 = S.weight(rw, H, F)
+    gamma = rw.uniform(0.5, 1.5, H).astype(np.float32)
+    beta = rw.normal(0, 0.1, H).astype(np.float32)
+    return {"x": S.to_bf16_bits(x), "dy": S.to_bf16_bits(dy), "w1": S.to_bf16_bits(w1), "w2": S.to_bf16_bits(w2),
+            "gamma": gamma, "beta": beta}
+
+
+def gpt2m_inputs(seed):
+    """GPT2-medium fc1 operands (M=4096, K=1024, N=4096; X with 10 channels x30) for the side measurements."""
+    from inputs import synthetic as S
+    w = S.WORKLOADS["gpt2m_fc1"]
+    M, K, N = w["M"], w["K"], w["N"]
+    rng = np.random.default_rng(seed)
     n_out, fac = w["x_outliers"]
     x = S.activation(rng, M, K, n_out, fac)
-    dy = S.grad(rng, M, N)
-    wt = S.weight(np.random.default_rng(seed_weight), N, K)
-    rng_ln = np.random.default_rng(seed_weight + 7)
-    gamma = rng_ln.uniform(0.5, 1.5, K).astype(np.float32)
-    beta = rng_ln.normal(0, 0.1, K).astype(np.float32)
-    return {"x": S.to_bf16_bits(x), "w": S.to_bf16_bits(wt), "dy": S.to_bf16_bits(dy), "gamma": gamma, "beta": beta}
+    wt = S.weight(np.random.default_rng(seed + 100), N, K)
+    return M, K, N, {"x": S.to_bf16_bits(x), "w": S.to_bf16_bits(wt)}
+
+
+def sbytes(r, c):
+    return (r // 32) * (c // 32) * 4
 
 
 def bytes_quant(r, c, in_bytes):  # read input, write codes + scales
-    return r * c * (in_bytes + 1) + (r // 32) * (c // 32) * 4
+    return r * c * (in_bytes + 1) + sbytes(r, c)
 
 
 def bytes_i8_op(r, c, extra=0):  # read codes + scales, write codes + scales
-    return 2 * (r * c + (r // 32) * (c // 32) * 4) + extra
+    return 2 * (r * c + sbytes(r, c)) + extra
 
 
 # --------------------------------------------------------------------------------------------
 # our implementation
 # --------------------------------------------------------------------------------------------
 class GpuStep:
-    OPS = ["quantize_x", "layernorm_i8", "quantize_w", "linear_fwd", "gelu_i8", "quantize_dy",
-           "linear_dgrad", "linear_wgrad", "dequantize_dx"]
+    OPS = ["quantize_x", "layernorm_i8", "quantize_w1", "quantize_w2", "fc1_fwd", "gelu_i8", "fc2_fwd",
+           "quantize_dy", "fc2_dgrad", "fc2_wgrad", "gelu_i8_bwd", "fc1_dgrad", "fc1_wgrad", "layernorm_i8_bwd",
+           "dequantize_dx"]
+    GEMMS = ["fc1_fwd", "fc2_fwd", "fc2_dgrad", "fc2_wgrad", "fc1_dgrad", "fc1_wgrad"]
 
-    def __init__(self, M, K, N, host, world_size):
+    def __init__(self, host, world_size):
         import torch
         import int8_fully_quantized_b200 as jf
         self.jf, self.torch = jf, torch
-        self.M, self.K, self.N, self.world = M, K, N, world_size
+        M, H, F = layer_dims()
+        self.M, self.H, self.F, self.world = M, H, F, world_size
         dev = torch.device("cuda", torch.cuda.current_device())
         bf = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
-        self.xb, self.wb, self.dyb = bf(host["x"]), bf(host["w"]), bf(host["dy"])
+        self.xb, self.dyb, self.w1b, self.w2b = bf(host["x"]), bf(host["dy"]), bf(host["w1"]), bf(host["w2"])
         self.gamma = torch.from_numpy(host["gamma"]).to(dev)
         self.beta = torch.from_numpy(host["beta"]).to(dev)
         e = lambda r, c: jf.empty_qtensor(r, c, dev)
-        self.Xq, self.Xn, self.Wq, self.Y, self.G = e(M, K), e(M, K), e(N, K), e(M, N), e(M, N)
-        self.dYq, self.dX, self.dW = e(M, N), e(M, K), e(N, K)
-        self.dx_bf16 = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
-        self.dw_f32 = torch.empty((N, K), dtype=torch.float32, device=dev) if world_size > 1 else None
-        self.launches_per_step = 9 + (1 if world_size > 1 else 0)
+        self.Xq, self.Xn, self.W1, self.W2 = e(M, H), e(M, H), e(F, H), e(H, F)
+        self.Y1, self.G, self.Y2 = e(M, F), e(M, F), e(M, H)
+        self.dY2, self.dG, self.dW2, self.dY1, self.dXn, self.dW1, self.dX = \
+            e(M, H), e(M, F), e(H, F), e(M, F), e(M, H), e(F, H), e(M, H)
+        self.dgamma = torch.empty(H, dtype=torch.float32, device=dev)
+        self.dbeta = torch.empty(H, dtype=torch.float32, device=dev)
+        self.ln_ws = torch.empty(jf.jf_layernorm_i8_bwd_workspace_bytes(M, H), dtype=torch.uint8, device=dev)
+        self.dx_bf16 = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+        if world_size > 1:
+            self.dw1_f32 = torch.empty((F, H), dtype=torch.float32, device=dev)
+            self.dw2_f32 = torch.empty((H, F), dtype=torch.float32, device=dev)
+        self.launches_per_step = (16 if world_size == 1 else 19)   # kernels of ours (LN backward: two)
         self.bytes = {
-            "quantize_x": bytes_quant(M, K, 2), "quantize_w": bytes_quant(N, K, 2), "quantize_dy": bytes_quant(M, N, 2),
-            "layernorm_i8": bytes_i8_op(M, K, 8 * K), "gelu_i8": bytes_i8_op(M, N),
-            "dequantize_dx": M * K * 3 + (M // 32) * (K // 32) * 4,
+            "quantize_x": bytes_quant(M, H, 2), "quantize_w1": bytes_quant(F, H, 2),
+            "quantize_w2": bytes_quant(H, F, 2), "quantize_dy": bytes_quant(M, H, 2),
+            "layernorm_i8": bytes_i8_op(M, H, 8 * H), "gelu_i8": bytes_i8_op(M, F),
+            "gelu_i8_bwd": bytes_i8_op(M, F, M * F + sbytes(M, F)),
+            "layernorm_i8_bwd": bytes_i8_op(M, H, M * H + sbytes(M, H) + 12 * H),
+            "dequantize_dx": M * H * 3 + sbytes(M, H),
         }
-        self.ops = {"linear_fwd": 2 * M * N * K, "linear_dgrad": 2 * M * K * N, "linear_wgrad": 2 * N * K * M}
+        self.ops = {g: 2 * M * H * F for g in self.GEMMS}
         self.side = torch.cuda.Stream(device=dev)
-        self.w_ready, self.dy_ready, self.xn_ready = torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event()
+        self.ev = {k: torch.cuda.Event() for k in ("w1", "w2", "dy", "g", "dy1")}
         self.graph = None
 
+    # the operators, one call each (the weight gradients in fp32 for the data-parallel sum)
+    def _op(self, name):
+        jf = self.jf
+        if name == "quantize_x": jf.jf_quantize_block(self.xb, self.Xq.q, self.Xq.s)
+        elif name == "layernorm_i8": jf.jf_layernorm_i8(self.Xq, self.gamma, self.beta, 1e-5, self.Xn)
+        elif name == "quantize_w1": jf.jf_quantize_block(self.w1b, self.W1.q, self.W1.s)
+        elif name == "quantize_w2": jf.jf_quantize_block(self.w2b, self.W2.q, self.W2.s)
+        elif name == "fc1_fwd": jf.jf_linear_fwd(self.Xn, self.W1, self.Y1)
+        elif name == "gelu_i8": jf.jf_gelu_i8(self.Y1, self.G)
+        elif name == "fc2_fwd": jf.jf_linear_fwd(self.G, self.W2, self.Y2)
+        elif name == "quantize_dy": jf.jf_quantize_block(self.dyb, self.dY2.q, self.dY2.s)
+        elif name == "fc2_dgrad": jf.jf_linear_dgrad(self.dY2, self.W2, self.dG)
+        elif name == "fc2_wgrad":
+            if self.world > 1: jf.jf_linear_wgrad(self.dY2, self.G, None, self.dw2_f32)
+            else: jf.jf_linear_wgrad(self.dY2, self.G, self.dW2)
+        elif name == "gelu_i8_bwd": jf.jf_gelu_i8_bwd(self.Y1, self.dG, self.dY1)
+        elif name == "fc1_dgrad": jf.jf_linear_dgrad(self.dY1, self.W1, self.dXn)
+        elif name == "fc1_wgrad":
+            if self.world > 1: jf.jf_linear_wgrad(self.dY1, self.Xn, None, self.dw1_f32)
+            else: jf.jf_linear_wgrad(self.dY1, self.Xn, self.dW1)
+        elif name == "layernorm_i8_bwd":
+            jf.jf_layernorm_i8_bwd(self.Xq, self.dXn, self.gamma, 1e-5, self.dX, self.dgamma, self.dbeta, self.ln_ws)
+        elif name == "dequantize_dx": jf.jf_dequantize_block(self.dX.q, self.dX.s, self.dx_bf16)
+        else: raise KeyError(name)
+
     def run_overlapped(self):
-        """The same nine operators on two streams, ordered by their data dependences only: quantize W
-        and quantize dY run beside quantize X and LayerNorm_i8, and the weight gradient (dY^T Xn)
-        needs neither the forward nor GELU, so it runs beside them and the input gradient; the
-        persistent GEMMs then fill each other's last partial wave of tiles."""
-        jf, t = self.jf, self.torch
+        """The step on two streams, ordered by its data dependences: the three bf16 quantizers of the
+        weights and the upstream gradient, and the two weight-gradient GEMMs, run on a side stream
+        beside the forward and the input-gradient chain (one GPU; captured as a CUDA graph)."""
+        t, ev = self.torch, self.ev
         main = t.cuda.current_stream()
         self.side.wait_stream(main)
         with t.cuda.stream(self.side):
-            jf.jf_quantize_block(self.wb, self.Wq.q, self.Wq.s)
-            self.w_ready.record()
-            jf.jf_quantize_block(self.dyb, self.dYq.q, self.dYq.s)
-            self.dy_ready.record()
-        jf.jf_quantize_block(self.xb, self.Xq.q, self.Xq.s)
-        jf.jf_layernorm_i8(self.Xq, self.gamma, self.beta, 1e-5, self.Xn)
-        self.xn_ready.record()
+            self._op("quantize_w1"); ev["w1"].record()
+            self._op("quantize_w2"); ev["w2"].record()
+            self._op("quantize_dy"); ev["dy"].record()
+        self._op("quantize_x")
+        self._op("layernorm_i8")
+        main.wait_event(ev["w1"])
+        self._op("fc1_fwd")
+        self._op("gelu_i8")
+        ev["g"].record()
+        main.wait_event(ev["w2"])
+        self._op("fc2_fwd")
+        main.wait_event(ev["dy"])
+        self._op("fc2_dgrad")
         with t.cuda.stream(self.side):
-            self.side.wait_event(self.xn_ready)
-            jf.jf_linear_wgrad(self.dYq, self.Xn, self.dW, None)
-        main.wait_event(self.w_ready)
-        jf.jf_linear_fwd(self.Xn, self.Wq, self.Y, None)
-        jf.jf_gelu_i8(self.Y, self.G)
-        main.wait_event(self.dy_ready)
-        jf.jf_linear_dgrad(self.dYq, self.Wq, self.dX, None)
-        jf.jf_dequantize_block(self.dX.q, self.dX.s, self.dx_bf16)
+            self.side.wait_event(ev["g"])
+            self._op("fc2_wgrad")
+        self._op("gelu_i8_bwd")
+        ev["dy1"].record()
+        self._op("fc1_dgrad")
+        with t.cuda.stream(self.side):
+            self.side.wait_event(ev["dy1"])
+            self._op("fc1_wgrad")
+        self._op("layernorm_i8_bwd")
+        self._op("dequantize_dx")
         main.wait_stream(self.side)
+
+    def run_data_parallel(self):
+        """The step on several ranks: each weight gradient is an fp32 partial over this rank's tokens;
+        its NCCL all-reduce is issued as soon as the partial exists and runs beside the rest of the
+        backward (WgradExchange); each summed gradient is re-quantized per block once its
+        all-reduce has landed."""
+        from int8_fully_quantized_b200.parallel import WgradExchange
+        ex = WgradExchange()
+        for op in ("quantize_x", "layernorm_i8", "quantize_w1", "quantize_w2", "fc1_fwd", "gelu_i8", "fc2_fwd",
+                   "quantize_dy", "fc2_dgrad", "fc2_wgrad"):
+            self._op(op)
+        ex.start(self.dw2_f32, self.dW2)
+        for op in ("gelu_i8_bwd", "fc1_dgrad", "fc1_wgrad"):
+            self._op(op)
+        ex.start(self.dw1_f32, self.dW1)
+        self._op("layernorm_i8_bwd")
+        self._op("dequantize_dx")
+        ex.finish(lambda dst, dw: self.jf.jf_quantize_block(dw, dst.q, dst.s))
+
+    def step(self):
+        if self.world > 1:
+            self.run_data_parallel()
+        elif self.graph is not None:
+            self.graph.replay()
+        else:
+            self.run_overlapped()
 
     def capture(self):
         """CUDA graph of run_overlapped (single GPU): one replay launches the step's kernels with no
@@ -239,34 +345,47 @@ class GpuStep:
         with t.cuda.graph(self.graph):
             self.run_overlapped()
 
-    def run(self, ev=None):
-        jf, t = self.jf, self.torch
-        mark = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
-        mark(0)
-        jf.jf_quantize_block(self.xb, self.Xq.q, self.Xq.s)
-        mark(1)
-        jf.jf_layernorm_i8(self.Xq, self.gamma, self.beta, 1e-5, self.Xn)
-        mark(2)
-        jf.jf_quantize_block(self.wb, self.Wq.q, self.Wq.s)
-        mark(3)
-        jf.jf_linear_fwd(self.Xn, self.Wq, self.Y, None)
-        mark(4)
-        jf.jf_gelu_i8(self.Y, self.G)
-        mark(5)
-        jf.jf_quantize_block(self.dyb, self.dYq.q, self.dYq.s)
-        mark(6)
-        jf.jf_linear_dgrad(self.dYq, self.Wq, self.dX, None)
-        mark(7)
-        if self.world > 1:
-            from int8_fully_quantized_b200.parallel import allreduce_wgrad_
-            jf.jf_linear_wgrad(self.dYq, self.Xn, None, self.dw_f32)
-            allreduce_wgrad_(self.dw_f32)
-            jf.jf_quantize_block(self.dw_f32, self.dW.q, self.dW.s)
-        else:
-            jf.jf_linear_wgrad(self.dYq, self.Xn, self.dW, None)
-        mark(8)
-        jf.jf_dequantize_block(self.dX.q, self.dX.s, self.dx_bf16)
-        mark(9)
+    def run_serialized(self, ev):
+        """Every operator on one stream, bracketed by events (the per-kernel times)."""
+        ev[0].record()
+        for i, op in enumerate(self.OPS):
+            self._op(op)
+            ev[i + 1].record()
+
+
+def _device_ms(fn, flush, reps=10):
+    """Median CUDA-event time of fn over reps launches, L2 flushed (256 MiB write) before each."""
+    import torch
+    for _ in range(3):
+        flush.zero_()
+        fn()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(); fn(); b.record()
+        ts.append((a, b))
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in ts)
+
+
+def tensor_ceiling(jf, flush, i8_peak):
+    """The plain INT8 product (jf_gemm_i8_s32: the same TMA / tcgen05 machinery, int32 result, no
+    per-block rescale) at the fc1 and fc2 shapes of the layer: the tensor core's measured INT8 rate."""
+    import torch
+    M, H, F = layer_dims()
+    g = torch.Generator(device="cuda").manual_seed(1)
+    out = {}
+    for name, (m, n, k) in (("fc1_shape", (M, F, H)), ("fc2_shape", (M, H, F))):
+        a = torch.randint(-127, 128, (m, k), dtype=torch.int8, device="cuda", generator=g)
+        b = torch.randint(-127, 128, (n, k), dtype=torch.int8, device="cuda", generator=g)
+        c = torch.empty((m, n), dtype=torch.int32, device="cuda")
+        ms = _device_ms(lambda: jf.jf_gemm_i8_s32(a, b, c), flush, reps=10)
+        tops = 2 * m * n * k / (ms * 1e-3) / 1e12
+        out[name] = {"M": m, "N": n, "K": k, "ms": round(ms, 4), "TOPS": round(tops, 1),
+                     "frac_of_peak": round(tops / i8_peak, 4), "frac_of_nominal_4500": round(tops / NOMINAL_I8_TOPS, 4)}
+        del a, b, c
+    return out
 
 
 def run_ours(args):
@@ -286,25 +405,22 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     jf.load_library()
-    wl = __import__("inputs.synthetic", fromlist=["WORKLOADS"]).WORKLOADS[WORKLOAD]
-    M, K, N = wl["M"], wl["K"], wl["N"]
-    host = host_inputs(M, K, N, P.shard_seed(0, rank), seed_weight=0)
-    step = GpuStep(M, K, N, host, world)
+    host = host_inputs(P.shard_seed(0, rank), seed_weight=0)
+    step = GpuStep(host, world)
     flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")   # 256 MiB > L2
-    stream = torch.cuda.current_stream()
 
     use_graph = world == 1 and not args.eager
     sampler = ClockSampler(local)
     with sampler:
         for _ in range(max(3, args.warmup)):
             flush.zero_()
-            step.run() if not use_graph else step.run_overlapped()
+            step.step()
         torch.cuda.synchronize()
         if use_graph:
             step.capture()
             for _ in range(max(3, args.warmup)):
                 flush.zero_()
-                step.graph.replay()
+                step.step()
         st = jf.jf_device_status()
         if st != 0:
             raise RuntimeError(f"device status after warm-up: {jf.jf_strerror(st)}")
@@ -313,85 +429,82 @@ def run_ours(args):
         torch.cuda.synchronize()
         # timed region: whole steps (graph replays on one GPU, eager launches on several)
         bounds = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(10)] for _ in range(args.steps)]
         for i in range(args.steps):
             flush.zero_()
-            if use_graph:
-                bounds[i][0].record()
-                step.graph.replay()
-                bounds[i][1].record()
-            else:
-                step.run(evs[i])
+            bounds[i][0].record()
+            step.step()
+            bounds[i][1].record()
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
         # per-kernel times: the operators serialized on one stream, each bracketed by events
-        n_ops = max(3, min(args.steps, 20))
-        op_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(10)] for _ in range(n_ops)] if use_graph else evs
-        if use_graph:
-            for i in range(n_ops):
-                flush.zero_()
-                step.run(op_evs[i])
-            torch.cuda.synchronize()
+        n_ops = max(3, min(args.steps, 5))
+        op_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(GpuStep.OPS) + 1)] for _ in range(n_ops)]
+        for i in range(n_ops):
+            flush.zero_()
+            step.run_serialized(op_evs[i])
+        torch.cuda.synchronize()
     st = jf.jf_device_status()
     if st != 0:
         raise RuntimeError(f"device status after the timed steps: {jf.jf_strerror(st)}")
-    per_op = {op: [op_evs[i][j].elapsed_time(op_evs[i][j + 1]) for i in range(len(op_evs))]
+    per_op = {op: [op_evs[i][j].elapsed_time(op_evs[i][j + 1]) for i in range(n_ops)]
               for j, op in enumerate(GpuStep.OPS)}
-    if use_graph:
-        step_ms_local = sum(a.elapsed_time(b) for a, b in bounds) / args.steps
-    else:
-        step_ms_local = sum(evs[i][0].elapsed_time(evs[i][9]) for i in range(args.steps)) / args.steps
+    step_ms_local = sum(a.elapsed_time(b) for a, b in bounds) / args.steps
     step_ms = P.max_over_ranks(step_ms_local, device="cuda")
     ops_per_step = sum(step.ops.values())
     value = world * ops_per_step / (step_ms * 1e-3) / 1e12
 
     peaks, peak_src = load_peaks()
-    i8_peak_burst = peaks["bf16_tflops"] * NOMINAL_I8_OVER_BF16
+    i8_peak = peaks["bf16_tflops"] * NOMINAL_I8_OVER_BF16
+    i8_peak_sustained = peaks["bf16_tflops_sustained"] * NOMINAL_I8_OVER_BF16
     kernels = {}
     for op, ts in per_op.items():
         ms = statistics.mean(ts)
         if op in step.ops:
             tops = step.ops[op] / (ms * 1e-3) / 1e12
-            kernels[op] = {"ms": round(ms, 4), "TOPS": round(tops, 1), "frac_i8_peak": round(tops / i8_peak_burst, 4)}
+            kernels[op] = {"ms": round(ms, 4), "TOPS": round(tops, 1), "frac_i8_peak": round(tops / i8_peak, 4)}
         else:
             gbs = step.bytes[op] / (ms * 1e-3) / 1e9
             kernels[op] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
-    gemm_ops = [op for op in step.ops]
-    dom = max(gemm_ops, key=lambda o: statistics.mean(per_op[o]))
+    dom = max(step.GEMMS, key=lambda o: statistics.mean(per_op[o]))
     dom_ms = statistics.mean(per_op[dom])
     achieved = step.ops[dom] / (dom_ms * 1e-3) / 1e12
-    traffic = _load_traffic(dom)
-    # The binding roofline of the block-scaled GEMM is the SM issue rate, not the tensor pipe: every
-    # output element needs, per 32-deep contraction block, an int32 -> fp32 convert and an FMA (two
-    # lane-instructions), i.e. M*N*K/16 per launch, and an SM issues at most 4 x 32 lane-instructions
-    # per clock. That ceiling (about 1.19 int8 POPS at 1965 MHz) lies below the tensor peak.
-    alu_work = step.ops[dom] // 32                      # 2*M*N*K / 32 = 2 instructions per (element, block)
-    alu_peak = ALU_LANES_PER_CLK_PER_SM * peaks.get("sm_count", B200_SMS) * peaks["sm_max_mhz"] * 1e6 / 1e12
+    # The same launch seen as issue work: per output element and 32-deep contraction block an int32 ->
+    # fp32 conversion and an FMA (M*N*K/16 lane-instructions per launch), against 4 x 32 lane-instructions
+    # per clock per SM: the CUDA-core ceiling of the per-block rescale.
+    alu_work = step.ops[dom] // 32
+    alu_peak = ALU_LANES_PER_CLK_PER_SM * B200_SMS * peaks["sm_max_mhz"] * 1e6 / 1e12
     alu_achieved = alu_work / (dom_ms * 1e-3) / 1e12
-    roofline = {"kernel": f"gemm_i8_kernel ({dom})", "bound": "alu", "achieved": round(alu_achieved, 2),
-                "peak": round(alu_peak, 2), "unit": "T lane-instructions/s", "frac": round(alu_achieved / alu_peak, 4),
-                "traffic": traffic,
-                "peak_source": f"{ALU_LANES_PER_CLK_PER_SM} lane-instructions/clk/SM (4 schedulers x 32 lanes) x "
-                               f"{B200_SMS} SMs x {peaks['sm_max_mhz']:g} MHz",
-                "algorithmic": f"2 per output element per 32-deep block = M*N*K/16 = {alu_work} per launch",
-                "tensor_view": {"achieved": round(achieved, 1), "peak": round(i8_peak_burst, 1), "unit": "TOPS",
-                                "frac": round(achieved / i8_peak_burst, 4),
-                                "peak_source": f"{peak_src} bf16 dense burst x {NOMINAL_I8_OVER_BF16:g}"}}
-
+    world_ok = world == 1
+    ceiling = tensor_ceiling(jf, flush, i8_peak) if world_ok else None
+    roofline = {"kernel": f"gemm_i8_kernel ({dom})", "bound": "tensor", "achieved": round(achieved, 1),
+                "peak": round(i8_peak, 1), "unit": "TOPS", "frac": round(achieved / i8_peak, 4),
+                "traffic": _load_traffic(dom),
+                "peak_source": f"{peak_src} bf16 dense burst {peaks['bf16_tflops']:g} TFLOP/s x nominal int8/bf16 "
+                               f"ratio {NOMINAL_I8_OVER_BF16:g}",
+                "algorithmic": f"2*M*N*K = {step.ops[dom]} int8 ops per launch (M=8192, N*K=4096*16384)",
+                "frac_of_sustained_peak": round(achieved / i8_peak_sustained, 4),
+                "frac_of_nominal_4500": round(achieved / NOMINAL_I8_TOPS, 4),
+                "measured_tensor_ceiling": ceiling,
+                "alu_view": {"achieved": round(alu_achieved, 2), "peak": round(alu_peak, 2),
+                             "unit": "T lane-instructions/s", "frac": round(alu_achieved / alu_peak, 4),
+                             "work": "2 per output element per 32-deep block = M*N*K/16 per launch",
+                             "peak_source": f"{ALU_LANES_PER_CLK_PER_SM} lane-instructions/clk/SM x {B200_SMS} SMs x "
+                                            f"{peaks['sm_max_mhz']:g} MHz (derived)"}}
+    M, H, F = step.M, step.H, step.F
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": round(step_ms, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
-        "config": {"workload": "GPT2-medium MLP fc1 linear fwd+dgrad+wgrad with quantize, LayerNorm_i8, GELU_i8 "
-                               "and dequantize (per rank)", "M": M, "K": K, "N": N, "block": 32,
-                   "inputs": "bf16 X ~N(0,1) with 10 channels x30, W ~N(0,0.02), dY ~N(0,1e-3)",
+        "config": {"workload": WORKLOAD_NAME, "M": M, "H": H, "F": F, "block": 32,
+                   "inputs": "bf16 X ~N(0,1) with 4 channels x50, W1, W2 ~N(0,0.02), dY ~N(0,1e-3)",
                    "parallelism": f"dp{world}", "l2": "flushed between steps (256 MiB write, outside timed events)"},
         "kernels": kernels, "roofline": roofline,
-        "execution": ("CUDA graph of the step on two streams ordered by data dependences (quantize W, quantize dY "
-                      "and the weight gradient beside quantize X, LayerNorm_i8, the forward, GELU_i8 and the input "
-                      "gradient); per-kernel times from the nine operators serialized on one stream"
-                      if use_graph else "eager launches on one stream, per-kernel events"),
+        "execution": ("CUDA graph of the step on two streams ordered by data dependences (the three bf16 quantizers "
+                      "of W1, W2, dY and the two weight-gradient GEMMs beside the forward and input-gradient chain); "
+                      "per-kernel times from the operators serialized on one stream"
+                      if use_graph else "eager launches; fp32 weight-gradient all-reduces (NCCL) overlap the rest "
+                                        "of the backward; per-kernel events serialized"),
         "gpu_launches": step.launches_per_step * args.steps,
         "clocks": sampler.summary(),
     }
@@ -400,9 +513,14 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+    if rank == 0 and world == 1:
+        del step
+        torch.cuda.empty_cache()
+        if not args.no_sweep:
+            result["sweep"] = memory_sweep(jf, [8192, 65536], SWEEP_OPS, flush, peaks)
+        if not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline(args.cpu_sample_blocks)
     if rank == 0:
-        if world == 1 and not args.no_cpu_baseline:
-            result["cpu_baseline"] = cpu_baseline(args.cpu_sample_tokens, host)
         print(json.dumps(result), flush=True)
 
 
@@ -423,24 +541,25 @@ def _load_traffic(kernel_op):
 
 
 def run_e2e(step, host, args, world, flush):
-    """Same step through the public API with host buffers. Every step copies its X, W and dY from
-    pinned host memory to the device, runs the nine operators, and reads dX (bf16) and dW (codes
-    and scales) back to pinned host memory. The steps are pipelined the way a training loop feeds
-    a GPU: two device input/output slots, the host->device copies of step i+1 on a copy stream and
-    the device->host reads of step i on a third stream while step i+1 computes. The timed window
-    runs from the first input copy to the last result read; ms_per_step = window / steps. The L2
-    flush before each step's operators is inside the window."""
+    """Same step through the public API with host buffers. Every step copies its batch (X and the
+    upstream gradient dY, bf16) from pinned host memory to the device, runs the layer's forward and
+    backward, and reads its results back to pinned host memory: dX (bf16), the re-quantized weight
+    gradients dW1, dW2 (codes and scales) and dgamma, dbeta. The weights are model state, resident
+    on the device. The steps are pipelined the way a training loop feeds a GPU: two device
+    input/output slots, the host->device copies of step i+1 on a copy stream and the device->host
+    reads of step i on a third stream while step i+1 computes. The timed window runs from the first
+    input copy to the last result read; ms_per_step = window / steps. The L2 flush before each
+    step's operators is inside the window."""
     import torch
     from int8_fully_quantized_b200 import parallel as P
     pin = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
-    hx, hw, hdy = pin(host["x"]), pin(host["w"]), pin(host["dy"])
-    out_dx = torch.empty(step.dx_bf16.shape, dtype=torch.bfloat16).pin_memory()
-    out_wq = torch.empty(step.dW.q.shape, dtype=torch.int8).pin_memory()
-    out_ws = torch.empty(step.dW.s.shape, dtype=torch.float32).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (hx, hw, hdy))
-    d2h = sum(t.numel() * t.element_size() for t in (out_dx, out_wq, out_ws))
+    hx, hdy = pin(host["x"]), pin(host["dy"])
+    outs = [step.dx_bf16, step.dW1.q, step.dW1.s, step.dW2.q, step.dW2.s, step.dgamma, step.dbeta]
+    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+    h2d = sum(t.numel() * t.element_size() for t in (hx, hdy))
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
 
-    slots = [step, GpuStep(step.M, step.K, step.N, host, world)]
+    slots = [step, GpuStep(host, world)]
     use_graph = world == 1 and not args.eager
     if use_graph:
         for s in slots:
@@ -461,7 +580,6 @@ def run_e2e(step, host, args, world, flush):
                 h2d_stream.wait_event(computed[k])   # step i-2 has finished reading this slot
             s = slots[k]
             s.xb.copy_(hx, non_blocking=True)
-            s.wb.copy_(hw, non_blocking=True)
             s.dyb.copy_(hdy, non_blocking=True)
             ready[k].record(h2d_stream)
 
@@ -472,16 +590,12 @@ def run_e2e(step, host, args, world, flush):
         if i >= 2:
             main.wait_event(read[k])   # step i-2's results have left this slot
         flush.zero_()
-        if use_graph:
-            s.graph.replay()
-        else:
-            s.run()
+        s.step()
         computed[k].record(main)
         with torch.cuda.stream(d2h_stream):
             d2h_stream.wait_event(computed[k])
-            out_dx.copy_(s.dx_bf16, non_blocking=True)
-            out_wq.copy_(s.dW.q, non_blocking=True)
-            out_ws.copy_(s.dW.s, non_blocking=True)
+            for dst, src in zip(host_out, [s.dx_bf16, s.dW1.q, s.dW1.s, s.dW2.q, s.dW2.s, s.dgamma, s.dbeta]):
+                dst.copy_(src, non_blocking=True)
             read[k].record(d2h_stream)
 
     def pipeline(n, started=None):
@@ -507,6 +621,7 @@ def run_e2e(step, host, args, world, flush):
     ms = t0.elapsed_time(t1) / args.steps
     ms = P.max_over_ranks(ms, device="cuda")
     ops = sum(step.ops.values())
+    del slots[1]
     return {"value": round(world * ops / (ms * 1e-3) / 1e12, 2), "unit": "TOPS", "ms_per_step": round(ms, 4),
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "pipelining": "two slots; step i+1's host->device copies and step i's device->host reads overlap the "
@@ -514,98 +629,21 @@ def run_e2e(step, host, args, world, flush):
 
 
 # --------------------------------------------------------------------------------------------
-# CPU oracle timings (the baseline leg, and the --impl reference arm)
+# memory-bound sweep (also reported in the main line at M = 8192 and 65536)
 # --------------------------------------------------------------------------------------------
-def _oracle_step(host, tokens):
-    """The whole step in the CPU oracle on the first `tokens` tokens of the batch (W in full).
-    Returns the GEMM int8 ops it performed."""
-    import oracle as O
-    K = host["x"].shape[1]
-    N = host["w"].shape[0]
-    x = O.bf16_bits_to_f32(host["x"][:tokens])
-    w = O.bf16_bits_to_f32(host["w"])
-    dy = O.bf16_bits_to_f32(host["dy"][:tokens])
-    Xq, Xs = O.quantize_block(x)
-    Xn_q, Xn_s, _ = O.layernorm_i8(Xq, Xs, host["gamma"], host["beta"], 1e-5)
-    Wq, Ws = O.quantize_block(w)
-    Y = O.linear_fwd(Xn_q, Xn_s, Wq, Ws)
-    Yq, Ys = O.requantize(Y)
-    O.gelu_i8(Yq, Ys)
-    dYq, dYs = O.quantize_block(dy)
-    dX = O.linear_dgrad(dYq, dYs, Wq, Ws)
-    dXq, dXs = O.requantize(dX)
-    O.requantize(O.linear_wgrad(dYq, dYs, Xn_q, Xn_s))
-    O.dequantize_block(dXq, dXs, "bf16")
-    return 3 * 2 * tokens * N * K
+SWEEP_OPS = ["quantize_bf16", "dequantize_bf16", "gelu_i8", "layernorm_i8", "gelu_i8_bwd", "layernorm_i8_bwd"]
 
 
-def _cpu_cores():
-    try:
-        from threadpoolctl import threadpool_info
-        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
-        return int(n)
-    except Exception:
-        return os.cpu_count() or 1
-
-
-def cpu_baseline(tokens, host):
-    t0 = time.perf_counter()
-    ops = _oracle_step(host, tokens)
-    dt = time.perf_counter() - t0
-    return {"value": round(ops / dt / 1e12, 6), "unit": "TOPS", "cores": _cpu_cores(), "kind": "oracle",
-            "seconds": round(dt, 2),
-            "sample": f"one oracle step on the first {tokens} of the 4096 tokens (full W), GEMM int8 ops / wall time"}
-
-
-def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
-        return
-    wl = __import__("inputs.synthetic", fromlist=["WORKLOADS"]).WORKLOADS[WORKLOAD]
-    M, K, N = wl["M"], wl["K"], wl["N"]
-    host = host_inputs(M, K, N, 1, seed_weight=0)
-    tokens = 256
-    for _ in range(max(3, args.warmup)):
-        _oracle_step(host, tokens)
-    times = []
-    ops = 0
-    for _ in range(args.steps):
-        t0 = time.perf_counter()
-        ops = _oracle_step(host, tokens)
-        times.append(time.perf_counter() - t0)
-    ms = 1e3 * sum(times) / len(times)
-    value = ops / (ms * 1e-3) / 1e12
-    cores = _cpu_cores()
-    line = {
-        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TOPS", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
-        "config": {"workload": "GPT2-medium MLP fc1 linear fwd+dgrad+wgrad with quantize, LayerNorm_i8, GELU_i8 "
-                               "and dequantize", "M": M, "K": K, "N": N, "block": 32, "parallelism": "oracle on host"},
-        "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": cores, "kind": "oracle",
-                         "sample": f"each step: the oracle's full step on the first {tokens} of the {M} tokens"},
-        "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-    }
-    print(json.dumps(line), flush=True)
-
-
-def run_sweep(args):
-    """Memory-bound sweep: quantize (bf16 in), dequantize (bf16 out), GELU_i8, LayerNorm_i8 and their
-    INT8 backward on M x 4096 tensors, M in {1024, 8192, 65536}; N(0,1) with 1% of the channels x100.
-    One JSON line with GB/s (algorithmic bytes: every input read once, every output written once)
-    and the fraction of the measured HBM copy bandwidth per kernel and size. With "fused_fc1" it
-    also times the GPT2-medium fc1 forward with GELU fused into the GEMM epilogue against the
-    forward GEMM followed by GELU_i8."""
+def memory_sweep(jf, ms_list, op_names, flush, peaks, reps=10):
+    """quantize (bf16 in), dequantize (bf16 out), GELU_i8, LayerNorm_i8 and their INT8 backward on
+    M x 4096 tensors, N(0,1) with 1% of the channels x100. GB/s from algorithmic bytes (every input
+    read once, every output written once) over the median CUDA-event time, L2 flushed before each
+    launch, and the fraction of the measured HBM copy bandwidth."""
     import torch
-    import int8_fully_quantized_b200 as jf
     from inputs import synthetic as S
-    torch.cuda.set_device(0)
-    jf.load_library()
-    peaks, peak_src = load_peaks()
-    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
     H = 4096
     out = {}
-    for M in args.sweep_m:
+    for M in ms_list:
         x = S.to_bf16_bits(S.memory_sweep_input(0, M, H))
         xb = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
         del x
@@ -616,34 +654,40 @@ def run_sweep(args):
         yb = torch.empty((M, H), dtype=torch.bfloat16, device="cuda")
         gamma = torch.ones(H, device="cuda")
         beta = torch.zeros(H, device="cuda")
-        ops = {
-            "quantize_bf16": (lambda: jf.jf_quantize_block(xb, Y.q, Y.s), bytes_quant(M, H, 2)),
-            "dequantize_bf16": (lambda: jf.jf_dequantize_block(Q.q, Q.s, yb), M * H * 3 + (M // 32) * (H // 32) * 4),
-            "gelu_i8": (lambda: jf.jf_gelu_i8(Q, Y), bytes_i8_op(M, H)),
-            "layernorm_i8": (lambda: jf.jf_layernorm_i8(Q, gamma, beta, 1e-5, Y), bytes_i8_op(M, H, 8 * H)),
-            "gelu_i8_bwd": (lambda: jf.jf_gelu_i8_bwd(Q, D, Y), bytes_i8_op(M, H, M * H + (M // 32) * (H // 32) * 4)),
-            "layernorm_i8_bwd": (lambda: jf.jf_layernorm_i8_bwd(Q, D, gamma, 1e-5, Y, dgam, dbet, ws),
-                                 bytes_i8_op(M, H, M * H + (M // 32) * (H // 32) * 4 + 12 * H)),
-        }
         dgam, dbet = torch.empty(H, device="cuda"), torch.empty(H, device="cuda")
         ws = torch.empty(jf.jf_layernorm_i8_bwd_workspace_bytes(M, H), dtype=torch.uint8, device="cuda")
+        ops = {
+            "quantize_bf16": (lambda: jf.jf_quantize_block(xb, Y.q, Y.s), bytes_quant(M, H, 2)),
+            "dequantize_bf16": (lambda: jf.jf_dequantize_block(Q.q, Q.s, yb), M * H * 3 + sbytes(M, H)),
+            "gelu_i8": (lambda: jf.jf_gelu_i8(Q, Y), bytes_i8_op(M, H)),
+            "layernorm_i8": (lambda: jf.jf_layernorm_i8(Q, gamma, beta, 1e-5, Y), bytes_i8_op(M, H, 8 * H)),
+            "gelu_i8_bwd": (lambda: jf.jf_gelu_i8_bwd(Q, D, Y), bytes_i8_op(M, H, M * H + sbytes(M, H))),
+            "layernorm_i8_bwd": (lambda: jf.jf_layernorm_i8_bwd(Q, D, gamma, 1e-5, Y, dgam, dbet, ws),
+                                 bytes_i8_op(M, H, M * H + sbytes(M, H) + 12 * H)),
+        }
         for name, (fn, nbytes) in ops.items():
-            if name not in args.sweep_ops:
+            if name not in op_names:
                 continue
-            for _ in range(3):
-                flush.zero_()
-                fn()
-            ts = []
-            for _ in range(max(5, args.steps // 5)):
-                flush.zero_()
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(); fn(); b.record()
-                ts.append((a, b))
-            torch.cuda.synchronize()
-            ms = statistics.median(a.elapsed_time(b) for a, b in ts)
+            ms = _device_ms(fn, flush, reps=reps)
             gbs = nbytes / (ms * 1e-3) / 1e9
             out[f"{name}@M={M}"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
         del xb, Q, D, Y, yb, ws
+        torch.cuda.empty_cache()
+    assert jf.jf_device_status() == 0
+    return out
+
+
+def run_sweep(args):
+    """The memory-bound sweep at M in {1024, 8192, 65536} (one JSON line); with "fused_fc1",
+    "granularity_mse" and "mxfp8_fc1" also the f1 fused epilogue, the f3 granularity MSEs and the f4
+    MXFP8 comparison on the GPT2-medium fc1 shapes."""
+    import torch
+    import int8_fully_quantized_b200 as jf
+    torch.cuda.set_device(0)
+    jf.load_library()
+    peaks, peak_src = load_peaks()
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    out = memory_sweep(jf, args.sweep_m, args.sweep_ops, flush, peaks, reps=max(5, args.steps // 5))
     if "fused_fc1" in args.sweep_ops:
         out.update(_sweep_fused_fc1(jf, flush))
     if "granularity_mse" in args.sweep_ops:
@@ -655,6 +699,108 @@ def run_sweep(args):
                       "l2": "flushed before every timed launch"}), flush=True)
 
 
+# --------------------------------------------------------------------------------------------
+# CPU oracle timings (the baseline leg, and the --impl reference arm)
+# --------------------------------------------------------------------------------------------
+_ORACLE_OPERANDS = {}
+
+
+def _oracle_operands():
+    """Quantized operands of the layer's six GEMMs and one 32-token strip of its memory-bound operators,
+    drawn with the workload's distributions and quantized by the oracle itself (values do not change
+    the oracle's cost; none of them comes from the GPU). Cached: built once, outside any timing."""
+    if _ORACLE_OPERANDS:
+        return _ORACLE_OPERANDS
+    import oracle as O
+    from inputs import synthetic as S
+    M, H, F = layer_dims()
+    rng = np.random.default_rng(3)
+    q = lambda a: O.quantize_block(a)
+    X = q(S.activation(rng, M, H, 4, 50.0))      # Xn stand-in [M, H]
+    G = q(S.activation(rng, M, F, 0, 1.0))       # GELU output stand-in [M, F]
+    W1, W2 = q(S.weight(rng, F, H)), q(S.weight(rng, H, F))
+    dY2, dY1 = q(S.grad(rng, M, H)), q(S.grad(rng, M, F))
+    _ORACLE_OPERANDS.update(
+        gemms=[("fc1_fwd", O.linear_fwd, X, W1, M, F), ("fc2_fwd", O.linear_fwd, G, W2, M, H),
+               ("fc2_dgrad", O.linear_dgrad, dY2, W2, M, F), ("fc2_wgrad", O.linear_wgrad, dY2, G, H, F),
+               ("fc1_dgrad", O.linear_dgrad, dY1, W1, M, H), ("fc1_wgrad", O.linear_wgrad, dY1, X, F, H)],
+        strip_x=S.activation(rng, 32, H, 4, 50.0), strip_dy=S.grad(rng, 32, H), strip_g=S.activation(rng, 32, F, 0, 1.0),
+        gamma=np.ones(H, np.float32), beta=np.zeros(H, np.float32), H=H, F=F)
+    return _ORACLE_OPERANDS
+
+
+def _oracle_sample(nblk, seed=0):
+    """The oracle on a bounded sample of one step: nblk x nblk output blocks (evenly spread) of each of
+    the six GEMMs with their full contraction, plus quantize, LayerNorm_i8 and its backward, GELU_i8
+    and its backward and dequantize on one 32-token strip. Returns (GEMM int8 ops done, seconds)."""
+    import oracle as O
+    d = _oracle_operands()
+    t0 = time.perf_counter()
+    ops = 0
+    for _, fn, A, B, rows, cols in d["gemms"]:
+        rb = list(np.linspace(0, rows // 32 - 1, nblk).astype(int))
+        cb = list(np.linspace(0, cols // 32 - 1, nblk).astype(int))
+        O.requantize(fn(*A, *B, rb, cb))
+        depth = A[0].shape[1] if fn is not O.linear_wgrad else A[0].shape[0]
+        ops += 2 * (32 * nblk) * (32 * nblk) * depth
+    xq, xs = O.quantize_block(d["strip_x"])
+    O.layernorm_i8(xq, xs, d["gamma"], d["beta"], 1e-5)
+    dq, ds = O.quantize_block(d["strip_dy"])
+    O.layernorm_i8_bwd(xq, xs, dq, ds, d["gamma"], 1e-5)
+    gq, gs = O.quantize_block(d["strip_g"])
+    O.gelu_i8(gq, gs)
+    O.gelu_i8_bwd(gq, gs, gq, gs)
+    O.dequantize_block(xq, xs, "bf16")
+    return ops, time.perf_counter() - t0
+
+
+def _cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(nblk):
+    _oracle_operands()
+    ops, dt = _oracle_sample(nblk)
+    return {"value": round(ops / dt / 1e12, 6), "unit": "TOPS", "cores": _cpu_cores(), "kind": "oracle",
+            "seconds": round(dt, 2),
+            "sample": f"{nblk}x{nblk} output blocks of each of the six GEMMs (full contraction) plus one 32-token "
+                      f"strip of every memory-bound operator; GEMM int8 ops done / wall time"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    nblk = 6
+    _oracle_operands()
+    for _ in range(max(3, args.warmup)):
+        _oracle_sample(nblk)
+    times, ops = [], 0
+    for _ in range(args.steps):
+        ops, dt = _oracle_sample(nblk)
+        times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    value = ops / (ms * 1e-3) / 1e12
+    cores = _cpu_cores()
+    M, H, F = layer_dims()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAME, "M": M, "H": H, "F": F, "block": 32, "parallelism": "oracle on host"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {nblk}x{nblk} output blocks of each of the six GEMMs (full "
+                                   f"contraction) plus one 32-token strip of every memory-bound operator"},
+        "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def _mxfp8_vs_int8(jf, flush):
     """The GPT2-medium fc1 forward (M=4096, K=1024, N=4096, bf16 inputs) two ways: Jetfire's 32x32
     INT8 blocks (quantize X and W, block-scaled INT8 GEMM with fp32 output) and MXFP8 (1x32 E8M0
@@ -662,9 +808,7 @@ def _mxfp8_vs_int8(jf, flush):
     launch) and the relative Frobenius error of each fp32 output against the exact product of the
     bf16 inputs (fp64 on the host)."""
     import torch
-    wl = __import__("inputs.synthetic", fromlist=["WORKLOADS"]).WORKLOADS[WORKLOAD]
-    M, K, N = wl["M"], wl["K"], wl["N"]
-    host = host_inputs(M, K, N, 0, seed_weight=0)
+    M, K, N, host = gpt2m_inputs(0)
     xb = torch.from_numpy(host["x"].view(np.int16)).cuda().view(torch.bfloat16)
     wb = torch.from_numpy(host["w"].view(np.int16)).cuda().view(torch.bfloat16)
     ref = (xb.cpu().double().numpy() @ wb.cpu().double().numpy().T)
@@ -706,8 +850,7 @@ def _granularity_mse(jf):
     import torch
     from inputs import synthetic as S
     res = {}
-    wl = __import__("inputs.synthetic", fromlist=["WORKLOADS"]).WORKLOADS[WORKLOAD]
-    host = host_inputs(wl["M"], wl["K"], wl["N"], 0, seed_weight=0)
+    _, _, _, host = gpt2m_inputs(0)
     cases = {"gpt2m_fc1_X": torch.from_numpy(host["x"].view(np.int16)).cuda().view(torch.bfloat16),
              "sweep_8192x4096": torch.from_numpy(S.to_bf16_bits(S.memory_sweep_input(0, 8192, 4096)).view(np.int16))
              .cuda().view(torch.bfloat16)}
@@ -722,9 +865,7 @@ def _sweep_fused_fc1(jf, flush):
     """GPT2-medium fc1 forward (M=4096, K=1024, N=4096): GELU fused into the GEMM epilogue versus the
     forward GEMM followed by GELU_i8 (device time of each variant, L2 flushed before each)."""
     import torch
-    wl = __import__("inputs.synthetic", fromlist=["WORKLOADS"]).WORKLOADS[WORKLOAD]
-    M, K, N = wl["M"], wl["K"], wl["N"]
-    host = host_inputs(M, K, N, 0, seed_weight=0)
+    M, K, N, host = gpt2m_inputs(0)
     X = jf.quantize_block(torch.from_numpy(host["x"].view(np.int16)).cuda().view(torch.bfloat16))
     W = jf.quantize_block(torch.from_numpy(host["w"].view(np.int16)).cuda().view(torch.bfloat16))
     Y, G, P = jf.empty_qtensor(M, N), jf.empty_qtensor(M, N), jf.empty_qtensor(M, N)
@@ -748,22 +889,6 @@ def _sweep_fused_fc1(jf, flush):
         ms = statistics.median(a.elapsed_time(b) for a, b in ts)
         res[name] = {"ms": round(ms, 4), "TOPS": round(2 * M * N * K / (ms * 1e-3) / 1e12, 1)}
     return res
-
-
-def _device_ms(fn, flush, reps=10):
-    """Median CUDA-event time of fn over reps launches, L2 flushed (256 MiB write) before each."""
-    import torch
-    for _ in range(3):
-        flush.zero_()
-        fn()
-    ts = []
-    for _ in range(reps):
-        flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(); fn(); b.record()
-        ts.append((a, b))
-    torch.cuda.synchronize()
-    return statistics.median(a.elapsed_time(b) for a, b in ts)
 
 
 def run_configs(args):

@@ -239,6 +239,18 @@ JF_API int jf_layernorm_i8_bwd_noalloc(jf_cqtensor X, jf_cqtensor dY, const floa
                                        jf_qtensor dX, float* dgamma, float* dbeta, void* stream);
 
 /*
+ * The plain INT8 tensor-core product C = A B^T with an int32 result and no scales (no counterpart
+ * on the pages: it measures the tensor core's INT8 rate, the ceiling the block-scaled GEMMs above
+ * are reported against, with the same TMA / tcgen05 machinery and no per-block rescale).
+ *   A  device int8 [M, K] row-major, B device int8 [N, K] row-major (both 16-byte aligned)
+ *   C  device int32 [M, N] row-major, 16-byte aligned (output), exact.
+ *   M a multiple of 128, N of 256, K of 128 and at most 65536 (no int32 overflow); else JF_ERR_SHAPE.
+ *   Errors: JF_ERR_NULL, JF_ERR_ALIGN, JF_ERR_ALIAS (C overlaps A or B) as elsewhere.
+ */
+JF_API int jf_gemm_i8_s32(const int8_t* A, const int8_t* B, int32_t* C, int64_t M, int64_t N, int64_t K,
+                          void* stream);
+
+/*
  * f3. Quantization at another granularity: the baselines of the summary's ablation ("Measured
  *     effects table": per-block scales quantize activations with channel outliers more accurately
  *     than per-token ones). The rule is that of jf_quantize_block (s = absmax / 127, IEEE quotient,

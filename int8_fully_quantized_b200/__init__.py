@@ -30,7 +30,7 @@ __all__ = [
     "jf_quantize_block_rowstats", "jf_layernorm_i8_rowstats", "quantize_block_rowstats", "layernorm_i8_rowstats",
     "jf_layernorm_i8_bwd_workspace_bytes", "jf_layernorm_i8_bwd_noalloc", "jf_quantize_granular",
     "jf_dequantize_granular", "jf_quantization_error", "jf_granular_scale_count", "jf_mx_quantize",
-    "jf_mx_linear_fwd", "jf_selftest_wait_timeout", "jf_strerror",
+    "jf_mx_linear_fwd", "jf_gemm_i8_s32", "jf_selftest_wait_timeout", "jf_strerror",
     "jf_device_status", "jf_sm_count",
     # allocating helpers
     "quantize_block", "dequantize_block", "linear_fwd", "linear_fwd_gelu", "linear_dgrad", "linear_wgrad",
@@ -47,7 +47,8 @@ EXPORTED_SYMBOLS = (
     "jf_linear_wgrad",
     "jf_gelu_i8", "jf_layernorm_i8", "jf_gelu_i8_bwd", "jf_layernorm_i8_bwd", "jf_layernorm_i8_bwd_workspace_bytes",
     "jf_layernorm_i8_bwd_noalloc", "jf_quantize_granular", "jf_dequantize_granular", "jf_quantization_error",
-    "jf_granular_scale_count", "jf_mx_quantize", "jf_mx_linear_fwd", "jf_selftest_wait_timeout", "jf_strerror",
+    "jf_granular_scale_count", "jf_mx_quantize", "jf_mx_linear_fwd", "jf_gemm_i8_s32", "jf_selftest_wait_timeout",
+    "jf_strerror",
     "jf_device_status",
     "jf_sm_count",
 )
@@ -102,6 +103,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.jf_granular_scale_count.argtypes = [i64, i64, i32]
     lib.jf_mx_quantize.argtypes = [vp, i32, i64, i64, vp, vp, vp]
     lib.jf_mx_linear_fwd.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp]
+    lib.jf_gemm_i8_s32.argtypes = [vp, vp, vp, i64, i64, i64, vp]
     lib.jf_selftest_wait_timeout.argtypes = [i64, vp]
     lib.jf_strerror.argtypes = [i32]
     lib.jf_strerror.restype = ctypes.c_char_p
@@ -326,6 +328,14 @@ def mx_linear_fwd(a_codes, a_scales, b_codes, b_scales, stream=None) -> torch.Te
     y = torch.empty((a_codes.shape[0], b_codes.shape[0]), dtype=torch.float32, device=a_codes.device)
     jf_mx_linear_fwd(a_codes, a_scales, b_codes, b_scales, y, stream)
     return y
+
+
+def jf_gemm_i8_s32(a: torch.Tensor, b: torch.Tensor, c: torch.Tensor, stream=None) -> None:
+    """c (int32 [M, N]) = a (int8 [M, K]) @ b (int8 [N, K])^T on the tensor core, no scales."""
+    lib = load_library()
+    M, K = a.shape
+    N = b.shape[0]
+    _check(lib.jf_gemm_i8_s32(_ptr(a), _ptr(b), _ptr(c), M, N, K, _stream(stream)), "jf_gemm_i8_s32")
 
 
 def jf_selftest_wait_timeout(limit_ns: int, stream=None) -> None:

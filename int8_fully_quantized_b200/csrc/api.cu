@@ -499,6 +499,22 @@ int jf_mx_linear_fwd(const uint8_t* a_codes, const uint8_t* a_scales, const uint
                                         static_cast<cudaStream_t>(stream)));
 }
 
+int jf_gemm_i8_s32(const int8_t* A, const int8_t* B, int32_t* C, int64_t M, int64_t N, int64_t K, void* stream) {
+  if (M < 0 || N < 0 || K < 0 || M % 128 != 0 || N % 256 != 0 || K % 128 != 0 || K > 65536 ||
+      M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31))
+    return JF_ERR_SHAPE;
+  if (M == 0 || N == 0) return JF_OK;
+  if (C == nullptr) return JF_ERR_NULL;
+  if (!aligned(C, 16)) return JF_ERR_ALIGN;
+  if (K == 0) return cuda_status(cudaMemsetAsync(C, 0, size_t(M * N * 4), static_cast<cudaStream_t>(stream)));
+  if (A == nullptr || B == nullptr) return JF_ERR_NULL;
+  if (!aligned(A, 16) || !aligned(B, 16)) return JF_ERR_ALIGN;
+  if (overlap(C, M * N * 4, A, M * K) || overlap(C, M * N * 4, B, N * K)) return JF_ERR_ALIAS;
+  const DevInfo d = device_info();
+  if (!d.ok) return JF_ERR_DEVICE;
+  return cuda_status(jf::launch_gemm_s32(A, B, C, M, N, K, d.status, d.sm_count, static_cast<cudaStream_t>(stream)));
+}
+
 int jf_selftest_wait_timeout(int64_t limit_ns, void* stream) {
   if (limit_ns < 1000000 || limit_ns > 10000000000ll) return JF_ERR_ARG;
   const DevInfo d = device_info();

@@ -1,5 +1,6 @@
 // Block-scaled INT8 GEMM on sm_100a tensor cores (tcgen05.mma kind::i8), used for the forward,
-// input-gradient and weight-gradient products of a Jetfire linear layer.
+// input-gradient and weight-gradient products of a Jetfire linear layer, and a plain INT8 GEMM with
+// an int32 result (the tensor-core ceiling the block-scaled one is measured against).
 //
 // Jetfire (atlas.scime.ai summary, "Approach"): linear operators read and write INT8 tensors with
 // one scale per 32x32 block, quantization is applied on-chip, and the weight gradient is also an
@@ -7,27 +8,38 @@
 // exact int32 partial P = sum_k A(r,k) B(c,k) is multiplied by c = fp32(sA(r/32,kb) * sB(c/32,kb))
 // and accumulated in fp32; after the last block the fp32 tile is re-quantized per 32x32 block.
 //
-// Design (one CTA per SM, persistent over 128 x 128 output tiles). Every barrier operation, TMA
-// issue and commit costs its issuing thread a few hundred cycles of latency, so the three pipeline
-// roles run in separate warps and overlap:
-//   warp 0       producer: lane 0 loads 128-byte-deep stages of A and B (TMA, 128-byte swizzle)
-//                into a 6-stage shared-memory ring; all 32 lanes copy the stage's 32 scales into
-//                the same slot (cp.async). A slot is refilled once the epilogue has finished the
-//                stage it held, which also means the MMAs that read it have completed.
-//   warp 1       MMA: lane 0 issues one tcgen05.mma (M=128, N=128, K=32) per 32-wide contraction
-//                block, each into a fresh int32 accumulator. The four 128-column TMEM accumulators
-//                form two groups of two: the MMAs of a group share one tcgen05.commit (each commit
-//                drains the tensor pipe) and the two groups double-buffer against the epilogue.
-//                Warp 1 also owns TMEM.
-//   warps 2-17   epilogue: warp w owns TMEM lanes 32 (w % 4) .. +31 and one 32-column block, i.e.
-//                exactly one 32x32 output block of the tile; four warps per SM sub-partition hide
-//                each other's TMEM load latency. Per contraction block a warp loads its 32 int32
-//                partials per thread (tcgen05.ld), converts them and accumulates fp32(sA*sB) * P in
-//                registers. After the last block it reduces the block's absmax across the warp and
-//                writes the 32x32 codes, the block scale and (optionally) the fp32 result.
+// Design of the block-scaled kernel (one CTA per SM, persistent over 128 x 128 output tiles). The
+// rescale needs, per output element and contraction block, an int32 -> fp32 conversion and an FMA
+// on the CUDA cores, four times the tensor core's time for the same block, so the kernel is built
+// to keep the epilogue warps busy without pause; the tensor core only has to stay ahead of them.
+// Each contraction block of a tile is one MMA into its own int32 TMEM accumulator; four such
+// accumulators (all 512 TMEM columns) rotate, so the MMAs run up to four blocks ahead:
+//   warp 0       producer: lane 0 loads 128-byte-deep stages of A and B (TMA, 128-byte swizzle,
+//                no multicast) into a 6-stage shared-memory ring; a slot is refilled once the MMAs
+//                that read it have completed (tcgen05.commit on the slot's `empty` barrier).
+//   warp 1       MMA: lane 0 issues one tcgen05.mma (M=128, N=128, K=32) per contraction block and
+//                commits it to that accumulator's `tfull` barrier. It reuses accumulator b as soon
+//                as all 8 epilogue warps have read it: they each bar.arrive on hardware barrier
+//                1 + b after their TMEM load, and warp 1 waits there with bar.sync (the only
+//                thread that waits on that hand-off), so no epilogue warp ever stalls on a release.
+//   warps 2-9    epilogue: warp w owns TMEM lanes 32 (w % 4) .. +31 and two 32-column blocks, i.e.
+//                two 32x32 output blocks of the tile. Per contraction block it waits for the
+//                accumulator's commit, loads its 64 int32 partials per thread (one tcgen05.ld),
+//                arrives on the hand-off barrier, and accumulates fp32(sA*sB) * P in registers
+//                (packed fma.rn.f32x2). The block scales come from global memory straight into
+//                registers, 32 contraction blocks per load (lane l holds block w0 + l), one window
+//                ahead, and are broadcast by warp shuffles. After the last block the warp reduces
+//                each block's absmax and writes its 32x32 codes, the block scale and (optionally)
+//                the fp32 result. Ten warps in all keep at most three on an SM sub-partition, so
+//                each thread may hold the 64 accumulators and 64 partials in registers.
 // Operand orientation: A and B are read K-major (contraction contiguous) or MN-major (output
 // index contiguous) straight from their row-major INT8 storage, so dgrad and wgrad re-block along
 // the other axis with no transpose pass.
+//
+// Every mbarrier wait is bounded (ptx.cuh). On a timeout the warp that saw it sets the CTA's abort
+// flag; every warp then stops waiting and computing but keeps its place in the hardware-barrier
+// hand-offs (one per contraction block, always in the same order), so those complete; in-flight
+// copies and MMAs are drained (bounded) before TMEM is freed.
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -43,23 +55,22 @@
 namespace jf {
 
 constexpr int BM = 128;             // tile rows = MMA M = TMEM lanes
-constexpr int BN = 128;             // tile cols = MMA N
+constexpr int BN = 128;             // tile cols = MMA N = TMEM columns of one accumulator
 constexpr int KB = 32;              // contraction block (one MMA, one rescale)
 constexpr int KBS = 4;              // contraction blocks per pipeline stage (128 bytes)
-constexpr int GRP = 2;              // contraction blocks per accumulator group (one commit)
+constexpr int NBUF = 4;             // TMEM accumulators (4 x 128 = all 512 columns)
 constexpr int STAGES = 6;
-constexpr int SC_FLOATS = 32;       // [row block r][kk] at r*4+kk, then [col block j][kk] at 16+j*4+kk
-constexpr int NUM_EPI_WARPS = 16;
+constexpr int NUM_EPI_WARPS = 8;    // each owns two 32x32 output blocks of the 128 x 128 tile
 constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
+constexpr uint32_t HANDOFF_THREADS = 32 * (NUM_EPI_WARPS + 1);   // epilogue warps + the MMA warp
 constexpr int A_STAGE = BM * KBS * KB;  // 16 KB
 constexpr int B_STAGE = BN * KBS * KB;  // 16 KB
-constexpr uint32_t TMEM_COLS = 2 * GRP * BN;   // two groups of two 128-column accumulators = 512
+constexpr uint32_t TMEM_COLS = NBUF * BN;
 
 constexpr int SMEM_A = 0;
 constexpr int SMEM_B = SMEM_A + STAGES * A_STAGE;
-constexpr int SMEM_SC = SMEM_B + STAGES * B_STAGE;
-constexpr int SMEM_BAR = SMEM_SC + STAGES * SC_FLOATS * 4;
-constexpr int NUM_BARS = 2 * STAGES + 4 + 1;
+constexpr int SMEM_BAR = SMEM_B + STAGES * B_STAGE;
+constexpr int NUM_BARS = 2 * STAGES + NBUF + 1;
 constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
 constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;  // + slack to align the base to 1024
 
@@ -83,10 +94,10 @@ struct __align__(64) GemmParams {
 };
 
 // tcgen05 instruction descriptor: s32 accumulator, signed int8 A and B, A/B major-ness, N, M.
-template <bool A_MN, bool B_MN>
+template <bool A_MN, bool B_MN, int N>
 __device__ constexpr uint32_t instr_desc() {
   return (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(A_MN) << 15) | (uint32_t(B_MN) << 16) |
-         (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+         (uint32_t(N >> 3) << 17) | (uint32_t(BM >> 4) << 24);
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 descriptor version.
@@ -111,40 +122,44 @@ __device__ __forceinline__ void store_block_q(const float (&acc)[32], int8_t* q,
   if (lane == 0) *s = bq.s;
 }
 
+// The 32 scales of one operand's row (or column) block `blk` for contraction blocks w0 .. w0+31:
+// lane l returns the scale of block w0 + l (0 past the end of the matrix or of the contraction).
+__device__ __forceinline__ float scale_window(const float* __restrict__ base, int64_t s_blk, int64_t s_k, int blk,
+                                              int nblk, int w0, int kblocks, int lane) {
+  const int kb = w0 + lane;
+  return (blk < nblk && kb < kblocks) ? __ldg(base + blk * s_blk + int64_t(kb) * s_k) : 0.0f;
+}
+
 template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem + SMEM_A;
   uint8_t* sB = smem + SMEM_B;
-  float* sSc = reinterpret_cast<float*>(smem + SMEM_SC);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SMEM_BAR);  // per stage: A, B and scales landed
-  uint64_t* empty = full + STAGES;      // per stage: the epilogue is done with the stage
-  uint64_t* tfull = empty + STAGES;     // per accumulator group: its MMAs completed
-  uint64_t* tempty = tfull + 2;         // per accumulator group: every epilogue warp has read it
-  uint64_t* drain = tempty + 2;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SMEM_BAR);  // per stage: A and B landed
+  uint64_t* empty = full + STAGES;      // per stage: the MMAs that read it completed
+  uint64_t* tfull = empty + STAGES;     // per accumulator: its MMA completed
+  uint64_t* drain = tfull + NBUF;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SMEM_MISC);
   volatile uint32_t* abort_flag = tmem_holder + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1 + 32);      // the TMA byte count plus one cp.async arrival per lane
-      mbar_init(&empty[s], NUM_EPI_WARPS);
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], NUM_EPI_WARPS);
-    }
+    for (int b = 0; b < NBUF; ++b) mbar_init(&tfull[b], 1);
     mbar_init(drain, 1);
     *abort_flag = 0u;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tensormap(&p.tma_a);
-    prefetch_tensormap(&p.tma_b);
-  }
-  if (warp == 1) {
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tensormap(&p.tma_a);
+      prefetch_tensormap(&p.tma_b);
+    }
+    __syncwarp();
     tmem_alloc(tmem_holder, TMEM_COLS);
     tmem_relinquish();
   }
@@ -153,173 +168,167 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_co
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  const int num_kstages = (p.kblocks + KBS - 1) / KBS;
+  const int kblocks = p.kblocks;
+  const int num_kstages = (kblocks + KBS - 1) / KBS;
   const int num_tiles = p.tiles_m * p.tiles_n;
   const int my_tiles = blockIdx.x < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
   const int total_stages = my_tiles * num_kstages;   // this CTA's stages, in order
+  const int total = my_tiles * kblocks;              // this CTA's contraction blocks, in order
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer warp
-    // Stage g goes to slot g % STAGES once the epilogue has finished the stage that held it (which
-    // also means the MMAs that read it have completed). Lane 0 loads A and B by TMA; every lane
-    // copies one of the stage's 32 scales (cp.async); the slot's full barrier counts both.
-    uint32_t pending = 0, pend_ph = 0;  // slots armed by lane 0, and the parity armed
-    for (int g = 0; g < total_stages; ++g) {
-      const int t = blockIdx.x + (g / num_kstages) * gridDim.x;
-      const int ks = g % num_kstages;
-      const int row0 = (t % p.tiles_m) * BM, col0 = (t / p.tiles_m) * BN;
-      const int kb0 = ks * KBS;
-      const int nk = min(KBS, p.kblocks - kb0);
-      const int st = g % STAGES;
-      const uint32_t ph = uint32_t(g / STAGES) & 1u;
-      if (!__all_sync(0xffffffffu, mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status))) break;
-      if (lane == 0) {
+    if (lane == 0) {
+      uint32_t pending = 0, pend_ph = 0;  // slots armed, and the parity armed
+      for (int g = 0; g < total_stages; ++g) {
+        const int t = blockIdx.x + (g / num_kstages) * gridDim.x;
+        const int ks = g % num_kstages;
+        const int row0 = (t % p.tiles_m) * BM, col0 = (t / p.tiles_m) * BN;
+        const int st = g % STAGES;
+        const uint32_t ph = uint32_t(g / STAGES) & 1u;
+        if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status)) break;
         mbar_arrive_expect_tx(&full[st], A_STAGE + B_STAGE);
         pending |= 1u << st;
         pend_ph = (pend_ph & ~(1u << st)) | (ph << st);
-        const int k0 = kb0 * KB;
+        const int k0 = ks * KBS * KB;
         if (!A_MN) tma_load_2d(sA + st * A_STAGE, &p.tma_a, &full[st], k0, row0);
         else tma_load_2d(sA + st * A_STAGE, &p.tma_a, &full[st], row0, k0);
         if (!B_MN) tma_load_2d(sB + st * B_STAGE, &p.tma_b, &full[st], k0, col0);
         else tma_load_2d(sB + st * B_STAGE, &p.tma_b, &full[st], col0, k0);
       }
-      // lane l < 16: A scale of row block l/4, block kk = l%4; lane l >= 16: B scale of col block (l-16)/4
-      const int kk = lane & 3, blk = (lane >> 2) & 3;
-      const bool is_a = lane < 16;
-      const int gb = is_a ? (row0 >> 5) + blk : (col0 >> 5) + blk;
-      const int nb = is_a ? (p.rows >> 5) : (p.cols >> 5);
-      if (kk < nk && gb < nb) {
-        const float* src = is_a ? p.a_s + gb * p.a_s_blk + int64_t(kb0 + kk) * p.a_s_k
-                                : p.b_s + gb * p.b_s_blk + int64_t(kb0 + kk) * p.b_s_k;
-        cp_async_4(sSc + st * SC_FLOATS + lane, src);
-      }
-      cp_async_mbar_arrive_noinc(&full[st]);
-    }
-    // Teardown: every copy issued has landed before the CTA exits.
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    if (lane == 0) {
+      // Teardown: every copy issued has landed before the CTA exits.
       for (int s = 0; s < STAGES; ++s)
         if (pending & (1u << s)) mbar_wait_teardown(&full[s], (pend_ph >> s) & 1u, p.status);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA warp
-    if (lane == 0) {
-      constexpr uint32_t idesc = instr_desc<A_MN, B_MN>();
-      uint32_t ngroups = 0;             // accumulator groups issued so far
-      bool issued = false;
-      bool ok = true;
-      for (int g = 0; ok && g < total_stages; ++g) {
-        const int st = g % STAGES;
-        const int nk = min(KBS, p.kblocks - (g % num_kstages) * KBS);
-        if (!mbar_wait(&full[st], uint32_t(g / STAGES) & 1u, abort_flag, p.status)) break;
+    constexpr uint32_t idesc = instr_desc<A_MN, B_MN, BN>();
+    // Position of the next contraction block to issue: tile-local block kb of the CTA's stage seq.
+    int it_kb = 0, it_stage = 0;
+    bool dead = false, issued = false;
+    // Issue the MMA of the next contraction block (in order) into accumulator `buf` (lane 0 only).
+    auto issue_next = [&](uint32_t buf) -> bool {
+      const int ks = it_kb / KBS, kk = it_kb % KBS;
+      const int slot = it_stage % STAGES;
+      if (kk == 0) {
+        if (!mbar_wait(&full[slot], uint32_t(it_stage / STAGES) & 1u, abort_flag, p.status)) return false;
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(sA + st * A_STAGE);
-        const uint32_t b_addr = smem_u32(sB + st * B_STAGE);
-        for (int k0 = 0; k0 < nk; k0 += GRP, ++ngroups) {
-          const uint32_t grp = ngroups & 1u, gph = (ngroups >> 1) & 1u;
-          if (!mbar_wait(&tempty[grp], gph ^ 1u, abort_flag, p.status)) { ok = false; break; }
-          tc_fence_after();
-          for (int kk = k0; kk < min(nk, k0 + GRP); ++kk) {
-            // K-major: the 32-byte K step moves inside the 128-byte swizzle row;
-            // MN-major: it moves by 32 rows of 128 bytes (four 8-row swizzle atoms).
-            const uint64_t ad = smem_desc(a_addr + (A_MN ? kk * 4096 : kk * 32), A_MN ? 16384 : 16, 1024);
-            const uint64_t bd = smem_desc(b_addr + (B_MN ? kk * 4096 : kk * 32), B_MN ? 16384 : 16, 1024);
-            mma_i8(tmem_base + (grp * GRP + uint32_t(kk - k0)) * BN, ad, bd, idesc, 0u);
-          }
-          tc_commit(&tfull[grp]);
-          issued = true;
-        }
       }
-      // Teardown: no MMA may still be writing TMEM when it is freed.
-      if (issued) {
-        tc_commit(drain);
-        mbar_wait_teardown(drain, 0u, p.status);
+      const uint32_t a_addr = smem_u32(sA + slot * A_STAGE);
+      const uint32_t b_addr = smem_u32(sB + slot * B_STAGE);
+      // K-major: the 32-byte K step moves inside the 128-byte swizzle row;
+      // MN-major: it moves by 32 rows of 128 bytes (four 8-row swizzle atoms).
+      const uint64_t ad = smem_desc(a_addr + (A_MN ? kk * 4096 : kk * 32), A_MN ? 16384 : 16, 1024);
+      const uint64_t bd = smem_desc(b_addr + (B_MN ? kk * 4096 : kk * 32), B_MN ? 16384 : 16, 1024);
+      mma_i8(tmem_base + buf * BN, ad, bd, idesc, 0u);
+      tc_commit(&tfull[buf]);
+      issued = true;
+      const int nk = min(KBS, kblocks - ks * KBS);
+      if (kk == nk - 1) {
+        tc_commit(&empty[slot]);   // the stage's last MMA: the slot may be refilled once it completes
+        ++it_stage;
       }
+      if (++it_kb == kblocks) it_kb = 0;
+      return true;
+    };
+    if (lane == 0) {
+      for (int g = 0; g < min(NBUF, total) && !dead; ++g) dead = !issue_next(uint32_t(g));
+    }
+    for (int g = 0; g < total; ++g) {
+      const uint32_t b = uint32_t(g) & (NBUF - 1);
+      named_bar_sync(1 + b, HANDOFF_THREADS);   // every epilogue warp has read accumulator b
+      if (lane == 0 && !dead && g + NBUF < total) {
+        tc_fence_after();
+        dead = !issue_next(b);
+      }
+      __syncwarp();
+    }
+    // Teardown: no MMA may still be writing TMEM when it is freed.
+    if (lane == 0 && issued) {
+      tc_commit(drain);
+      mbar_wait_teardown(drain, 0u, p.status);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ epilogue warps
-    const int sub = warp & 3;           // TMEM sub-partition this warp may access = row block in the tile
-    const int cblk = (warp - 2) >> 2;   // column block of the tile
-    const uint32_t t_base = tmem_base + (uint32_t(sub * 32) << 16) + uint32_t(cblk * 32);
-    uint32_t ngroups = 0;               // accumulator groups consumed so far
-    bool ok = true;
-    // Accumulate c * P from accumulator `buf`; `release` hands group `grp` back once its last
-    // accumulator is in registers.
-    auto kblock = [&](const uint32_t buf, const float c, float (&acc)[32], const bool release, const uint32_t grp) {
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(t_base + buf * BN, r);
-      tc_wait_ld(r);
-      if (release) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[grp]);
-      }
-#pragma unroll
-      for (int i = 0; i < 32; ++i) acc[i] = fmaf(c, __int2float_rn(int(r[i])), acc[i]);
+    const int sub = warp & 3;             // TMEM sub-partition this warp may access = row block in the tile
+    const int cb0 = ((warp - 2) >> 2) * 2;  // first of the warp's two column blocks in the tile
+    const uint32_t t_base = tmem_base + (uint32_t(sub * 32) << 16) + uint32_t(cb0 * 32);
+    const int nrb = p.rows >> 5, ncb = p.cols >> 5;
+    bool dead = false;
+    uint32_t g = 0;                       // contraction blocks consumed so far (accumulator g % NBUF)
+    // Scales of the current window (lane l: contraction block w0 + l) of the warp's row block (sa)
+    // and two column blocks (sb0, sb1); each window prefetches the next one.
+    float sa_n, sb0_n, sb1_n;
+    auto load_scales = [&](int t, int w0, bool valid) {
+      const int rbk = (t % p.tiles_m) * (BM / 32) + sub, cbk = (t / p.tiles_m) * (BN / 32) + cb0;
+      sa_n = scale_window(p.a_s, p.a_s_blk, p.a_s_k, rbk, valid ? nrb : 0, w0, kblocks, lane);
+      sb0_n = scale_window(p.b_s, p.b_s_blk, p.b_s_k, cbk, valid ? ncb : 0, w0, kblocks, lane);
+      sb1_n = scale_window(p.b_s, p.b_s_blk, p.b_s_k, cbk + 1, valid ? ncb : 0, w0, kblocks, lane);
     };
-    // Wait until accumulator group `grp` (phase gph) holds the next contraction blocks.
-    auto wait_group = [&](const uint32_t grp, const uint32_t gph) -> bool {
-      const bool good = mbar_try_wait(&tfull[grp], gph) || mbar_wait(&tfull[grp], gph, abort_flag, p.status);
-      if (!__all_sync(0xffffffffu, good)) return false;
-      tc_fence_after();
-      return true;
-    };
-    for (int g0 = 0; ok && g0 < total_stages; g0 += num_kstages) {
-      const int t = blockIdx.x + (g0 / num_kstages) * gridDim.x;
-      const int row0 = (t % p.tiles_m) * BM, col0 = (t / p.tiles_m) * BN;
-      float acc[32];
+    load_scales(blockIdx.x, 0, my_tiles > 0);
+    for (int tile = 0; tile < my_tiles; ++tile) {
+      const int t = blockIdx.x + tile * gridDim.x;
+      const int rbk = (t % p.tiles_m) * (BM / 32) + sub, cbk = (t / p.tiles_m) * (BN / 32) + cb0;
+      float acc[2][32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
-      for (int ks = 0; ok && ks < num_kstages; ++ks) {
-        const int g = g0 + ks;
-        const int st = g % STAGES;
-        const int nk = min(KBS, p.kblocks - ks * KBS);
-        const uint32_t sph = uint32_t(g / STAGES) & 1u;
-        ok = mbar_try_wait(&full[st], sph) || mbar_wait(&full[st], sph, abort_flag, p.status);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        const float* slot = sSc + st * SC_FLOATS;
-        const float4 sa = *reinterpret_cast<const float4*>(slot + sub * 4);
-        const float4 sb = *reinterpret_cast<const float4*>(slot + 16 + cblk * 4);
-        const float c0 = sa.x * sb.x, c1 = sa.y * sb.y, c2 = sa.z * sb.z, c3 = sa.w * sb.w;  // fp32(sA * sB)
-        {  // blocks 0 and 1 of the stage
-          const uint32_t grp = ngroups & 1u;
-          if (!(ok = wait_group(grp, (ngroups >> 1) & 1u))) break;
-          kblock(grp * GRP + 0, c0, acc, nk == 1, grp);
-          if (nk >= 2) kblock(grp * GRP + 1, c1, acc, true, grp);
-          ++ngroups;
+      for (int i = 0; i < 32; ++i) acc[0][i] = acc[1][i] = 0.0f;
+      for (int w0 = 0; w0 < kblocks; w0 += 32) {
+        const float sa = sa_n, sb0 = sb0_n, sb1 = sb1_n;
+        if (w0 + 32 < kblocks) load_scales(t, w0 + 32, true);   // the rest of this tile
+        else load_scales(t + gridDim.x, 0, tile + 1 < my_tiles);  // the start of the next one
+        const int nk = min(32, kblocks - w0);
+        for (int j = 0; j < nk; ++j, ++g) {
+          const uint32_t b = g & (NBUF - 1);
+          dead = dead || __any_sync(0xffffffffu, *abort_flag != 0u);
+          uint32_t r[64];
+          if (!dead) {
+            const uint32_t ph = (g / NBUF) & 1u;
+            const bool good = mbar_try_wait(&tfull[b], ph) || mbar_wait(&tfull[b], ph, abort_flag, p.status);
+            dead = !__all_sync(0xffffffffu, good);
+          }
+          if (!dead) {
+            tc_fence_after();
+            tmem_ld_32x32b_x64(t_base + b * BN, r);
+            tc_wait_ld64(r);
+          }
+          tc_fence_before();
+          named_bar_arrive(1 + b, HANDOFF_THREADS);   // accumulator b may be reused
+          // fp32(sA * sB) of contraction block w0 + j for the warp's two output blocks
+          const float a = __shfl_sync(0xffffffffu, sa, j);
+          const float c0 = a * __shfl_sync(0xffffffffu, sb0, j), c1 = a * __shfl_sync(0xffffffffu, sb1, j);
+          if (!dead) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              fma_x2(c0, c0, __int2float_rn(int(r[i])), __int2float_rn(int(r[i + 1])), acc[0][i], acc[0][i + 1],
+                     acc[0][i], acc[0][i + 1]);
+              fma_x2(c1, c1, __int2float_rn(int(r[32 + i])), __int2float_rn(int(r[33 + i])), acc[1][i],
+                     acc[1][i + 1], acc[1][i], acc[1][i + 1]);
+            }
+          }
         }
-        if (nk > GRP) {  // blocks 2 and 3
-          const uint32_t grp = ngroups & 1u;
-          if (!(ok = wait_group(grp, (ngroups >> 1) & 1u))) break;
-          kblock(grp * GRP + 0, c2, acc, nk == 3, grp);
-          if (nk == 4) kblock(grp * GRP + 1, c3, acc, true, grp);
-          ++ngroups;
-        }
-        // every accumulator of the stage has been read: its MMAs completed, the slot may be refilled
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);
       }
-      if (!ok) break;
 
-      // ---- on-chip re-quantization of this warp's 32x32 block
-      const int rbk = (row0 >> 5) + sub, cbk = (col0 >> 5) + cblk;
-      if (rbk < (p.rows >> 5) && cbk < (p.cols >> 5)) {
-        const int64_t off = (int64_t(rbk) * 32 + lane) * p.ld_y + int64_t(cbk) * 32;
-        const int64_t soff = int64_t(rbk) * (p.cols >> 5) + cbk;
+      // ---- on-chip re-quantization of this warp's two 32x32 blocks of the finished tile (the loop is
+      // unrolled so that acc stays in registers)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (dead || rbk >= nrb || cbk + h >= ncb) continue;
+        float (&y)[32] = acc[h];
+        const int64_t off = (int64_t(rbk) * 32 + lane) * p.ld_y + int64_t(cbk + h) * 32;
+        const int64_t soff = int64_t(rbk) * ncb + cbk + h;
         if (p.act == kActGelu) {
           // fused activation: the fp32 pre-activation is re-quantized (when asked for) and GELU is
           // applied to it on chip, so neither ever makes an HBM round trip in fp32
-          if (p.pre_q != nullptr) store_block_q(acc, p.pre_q + off, p.pre_s + soff, lane);
+          if (p.pre_q != nullptr) store_block_q(y, p.pre_q + off, p.pre_s + soff, lane);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) acc[i] = gelu_f32(acc[i]);
+          for (int i = 0; i < 32; ++i) y[i] = gelu_f32(y[i]);
         }
-        if (p.y_q != nullptr) store_block_q(acc, p.y_q + off, p.y_s + soff, lane);
+        if (p.y_q != nullptr) store_block_q(y, p.y_q + off, p.y_s + soff, lane);
         if (p.y_f32 != nullptr) {
           float4* dst = reinterpret_cast<float4*>(p.y_f32 + off);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+          for (int i = 0; i < 8; ++i) dst[i] = make_float4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
         }
       }
     }
@@ -328,7 +337,155 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_co
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+  if (warp == 0) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Plain INT8 GEMM, C (int32) = A B^T, for measuring the tensor core's INT8 rate: the same TMA and
+// tcgen05 machinery with the whole contraction accumulated in TMEM (no per-block rescale), tiles of
+// 128 x 256 (MMA N = 256), two 256-column accumulators so the epilogue of one tile overlaps the
+// MMAs of the next. Both operands K-major; M % 128 == 0, N % 256 == 0, K % 128 == 0.
+//   warp 0 producer (as above), warp 1 MMA, warps 2-9 epilogue (TMEM -> int32 rows in global).
+// ---------------------------------------------------------------------------------------------
+constexpr int S32_BN = 256;
+constexpr int S32_STAGES = 4;
+constexpr int S32_EPI_WARPS = 8;
+constexpr int S32_THREADS = 64 + 32 * S32_EPI_WARPS;
+constexpr int S32_A_STAGE = BM * KBS * KB;       // 16 KB
+constexpr int S32_B_STAGE = S32_BN * KBS * KB;   // 32 KB
+constexpr int S32_SMEM_BAR = S32_STAGES * (S32_A_STAGE + S32_B_STAGE);
+constexpr int S32_NUM_BARS = 2 * S32_STAGES + 4 + 1;
+constexpr int S32_SMEM_BYTES = S32_SMEM_BAR + S32_NUM_BARS * 8 + 16 + 1024;
+
+struct __align__(64) GemmS32Params {
+  CUtensorMap tma_a;
+  CUtensorMap tma_b;
+  int32_t* c;
+  int64_t ldc;
+  unsigned int* status;
+  int kblocks, tiles_m, tiles_n;
+};
+
+__global__ void __launch_bounds__(S32_THREADS, 1) gemm_i8_s32_kernel(const __grid_constant__ GemmS32Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S32_STAGES * S32_A_STAGE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S32_SMEM_BAR);
+  uint64_t* empty = full + S32_STAGES;
+  uint64_t* tfull = empty + S32_STAGES;   // per accumulator: the tile's MMAs completed
+  uint64_t* tempty = tfull + 2;           // per accumulator: every epilogue warp has read it
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile uint32_t* abort_flag = tmem_holder + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S32_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], S32_EPI_WARPS);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  const int num_kstages = p.kblocks / KBS;
+  const int num_tiles = p.tiles_m * p.tiles_n;
+  const int my_tiles = blockIdx.x < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const int total_stages = my_tiles * num_kstages;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t pending = 0, pend_ph = 0;
+      for (int g = 0; g < total_stages; ++g) {
+        const int t = blockIdx.x + (g / num_kstages) * gridDim.x;
+        const int k0 = (g % num_kstages) * KBS * KB;
+        const int row0 = (t % p.tiles_m) * BM, col0 = (t / p.tiles_m) * S32_BN;
+        const int st = g % S32_STAGES;
+        const uint32_t ph = uint32_t(g / S32_STAGES) & 1u;
+        if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status)) break;
+        mbar_arrive_expect_tx(&full[st], S32_A_STAGE + S32_B_STAGE);
+        pending |= 1u << st;
+        pend_ph = (pend_ph & ~(1u << st)) | (ph << st);
+        tma_load_2d(sA + st * S32_A_STAGE, &p.tma_a, &full[st], k0, row0);
+        tma_load_2d(sB + st * S32_B_STAGE, &p.tma_b, &full[st], k0, col0);
+      }
+      for (int s = 0; s < S32_STAGES; ++s)
+        if (pending & (1u << s)) mbar_wait_teardown(&full[s], (pend_ph >> s) & 1u, p.status);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = instr_desc<false, false, S32_BN>();
+      bool issued = false, ok = true;
+      int g = 0;
+      for (int i = 0; ok && i < my_tiles; ++i) {
+        const uint32_t buf = uint32_t(i) & 1u;
+        if (!mbar_wait(&tempty[buf], (uint32_t(i >> 1) & 1u) ^ 1u, abort_flag, p.status)) break;
+        tc_fence_after();
+        for (int ks = 0; ks < num_kstages; ++ks, ++g) {
+          const int st = g % S32_STAGES;
+          if (!mbar_wait(&full[st], uint32_t(g / S32_STAGES) & 1u, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + st * S32_A_STAGE), b_addr = smem_u32(sB + st * S32_B_STAGE);
+#pragma unroll
+          for (int kk = 0; kk < KBS; ++kk)
+            mma_i8(tmem_base + buf * S32_BN, smem_desc(a_addr + kk * 32, 16, 1024), smem_desc(b_addr + kk * 32, 16, 1024),
+                   idesc, (ks | kk) != 0 ? 1u : 0u);
+          tc_commit(&empty[st]);
+          issued = true;
+        }
+        if (ok) tc_commit(&tfull[buf]);
+      }
+      if (issued) {
+        tc_commit(drain);
+        mbar_wait_teardown(drain, 0u, p.status);
+      }
+    }
+    __syncwarp();
+  } else {
+    const int sub = warp & 3, half = (warp - 2) >> 2;
+    const uint32_t t_base = tmem_base + (uint32_t(sub * 32) << 16) + uint32_t(half * 128);
+    for (int i = 0; i < my_tiles; ++i) {
+      const uint32_t buf = uint32_t(i) & 1u;
+      const uint32_t ph = uint32_t(i >> 1) & 1u;
+      const bool good = mbar_try_wait(&tfull[buf], ph) || mbar_wait(&tfull[buf], ph, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, good)) break;
+      tc_fence_after();
+      const int t = blockIdx.x + i * gridDim.x;
+      const int64_t row = int64_t(t % p.tiles_m) * BM + sub * 32 + lane;
+      int32_t* dst = p.c + row * p.ldc + int64_t(t / p.tiles_m) * S32_BN + half * 128;
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_base + buf * S32_BN + ch * 32, r);
+        tc_wait_ld(r);
+        int4* d4 = reinterpret_cast<int4*>(dst + ch * 32);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) d4[j] = make_int4(int(r[4 * j]), int(r[4 * j + 1]), int(r[4 * j + 2]), int(r[4 * j + 3]));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem_base, 512);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -426,6 +583,35 @@ cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t st) {
   if (!a_mn && !b_mn) return run<false, false>(prm, grid, st);
   if (!a_mn && b_mn) return run<false, true>(prm, grid, st);
   return run<true, true>(prm, grid, st);
+}
+
+cudaError_t launch_gemm_s32(const int8_t* a, const int8_t* b, int32_t* c, int64_t M, int64_t N, int64_t K,
+                            unsigned int* status, int sm_count, cudaStream_t st) {
+  GemmS32Params prm;
+  memset(&prm, 0, sizeof(prm));
+  if (!make_map(&prm.tma_a, a, uint64_t(K), uint64_t(M), uint64_t(K), 128, BM) ||
+      !make_map(&prm.tma_b, b, uint64_t(K), uint64_t(N), uint64_t(K), 128, S32_BN))
+    return cudaErrorInvalidValue;
+  prm.c = c;
+  prm.ldc = N;
+  prm.status = status;
+  prm.kblocks = int(K / KB);
+  prm.tiles_m = int(M / BM);
+  prm.tiles_n = int(N / S32_BN);
+  const int tiles = prm.tiles_m * prm.tiles_n;
+  const int grid = tiles < sm_count ? tiles : sm_count;
+  static unsigned long long attr_set = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attr_set & bit)) {
+    e = cudaFuncSetAttribute(gemm_i8_s32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, S32_SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set |= bit;
+  }
+  gemm_i8_s32_kernel<<<grid, S32_THREADS, S32_SMEM_BYTES, st>>>(prm);
+  return cudaGetLastError();
 }
 
 }  // namespace jf

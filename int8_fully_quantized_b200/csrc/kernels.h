@@ -83,4 +83,9 @@ struct GemmArgs {
 
 cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t st);
 
+// Plain INT8 GEMM C = A B^T (int32), A [M, K] and B [N, K] row-major: the tensor core's INT8 rate with
+// no per-block rescale. M % 128 == 0, N % 256 == 0, K % 128 == 0.
+cudaError_t launch_gemm_s32(const int8_t* a, const int8_t* b, int32_t* c, int64_t M, int64_t N, int64_t K,
+                            unsigned int* status, int sm_count, cudaStream_t st);
+
 }  // namespace jf

@@ -27,6 +27,36 @@ def allreduce_wgrad_(dw_f32: torch.Tensor) -> torch.Tensor:
     return dw_f32
 
 
+class WgradExchange:
+    """Overlapped exchange of the fp32 weight-gradient partials of one data-parallel step.
+
+    ``start(dw_f32)`` issues the all-reduce of a partial as soon as its wgrad kernel has been
+    enqueued (asynchronously: NCCL runs it on its own stream, ordered after the wgrad, while the
+    caller enqueues the rest of the backward on the compute stream). ``finish(requantize)`` waits
+    for every started all-reduce, in the order they were started, and hands each summed partial to
+    ``requantize`` (the per-block quantizer of the caller's choice, e.g. ``jf_quantize_block`` into
+    the INT8 dW). On one rank there is nothing to sum: ``start`` only records the tensor.
+    Every rank must start the same tensors in the same order (the collectives pair up by order)."""
+
+    def __init__(self):
+        self._pending = []
+
+    def start(self, dw_f32: torch.Tensor, tag=None) -> None:
+        _, n = world()
+        handle = dist.all_reduce(dw_f32, op=dist.ReduceOp.SUM, async_op=True) if n > 1 else None
+        self._pending.append((tag, dw_f32, handle))
+
+    def finish(self, requantize) -> list:
+        """Wait for the all-reduces and re-quantize each sum; returns requantize's results in order."""
+        out = []
+        for tag, dw, handle in self._pending:
+            if handle is not None:
+                handle.wait()
+            out.append(requantize(tag, dw))
+        self._pending = []
+        return out
+
+
 def max_over_ranks(value: float, device=None) -> float:
     """Largest value of a per-rank measurement (a step time) across ranks."""
     _, n = world()

@@ -25,11 +25,28 @@ def test_alu_issue_peak():
 
 
 def test_step_inputs_are_seeded_and_shaped():
-    a = bench.host_inputs(64, 96, 128, seed_tokens=3, seed_weight=0)
-    b = bench.host_inputs(64, 96, 128, seed_tokens=3, seed_weight=0)
-    c = bench.host_inputs(64, 96, 128, seed_tokens=4, seed_weight=0)
-    assert a["x"].shape == (64, 96) and a["w"].shape == (128, 96) and a["dy"].shape == (64, 128)
+    dims = (64, 96, 128)
+    a = bench.host_inputs(3, 0, dims)
+    b = bench.host_inputs(3, 0, dims)
+    c = bench.host_inputs(4, 0, dims)
+    assert a["x"].shape == (64, 96) and a["dy"].shape == (64, 96)
+    assert a["w1"].shape == (128, 96) and a["w2"].shape == (96, 128)
     assert a["x"].dtype == np.uint16 and a["gamma"].shape == (96,) and a["beta"].shape == (96,)
     for k in a:
         assert np.array_equal(a[k], b[k])                       # same seeds, same inputs
-    assert not np.array_equal(a["x"], c["x"]) and np.array_equal(a["w"], c["w"])  # per-rank tokens, shared W
+    # per-rank tokens, shared weights
+    assert not np.array_equal(a["x"], c["x"]) and np.array_equal(a["w1"], c["w1"]) and np.array_equal(a["w2"], c["w2"])
+
+
+def test_step_covers_the_path_and_counts_six_gemms():
+    """One step runs every operator of the path (quantize, dequantize, LayerNorm_i8, GELU_i8, the
+    three GEMM modes of both linears, and the two INT8 backward operators), and its GEMM work is six
+    products of 2 * M * H * F int8 ops."""
+    ops = bench.GpuStep.OPS
+    for name in ("quantize_x", "dequantize_dx", "layernorm_i8", "gelu_i8", "fc1_fwd", "fc2_dgrad", "fc1_wgrad",
+                 "gelu_i8_bwd", "layernorm_i8_bwd"):
+        assert name in ops
+    assert sorted(bench.GpuStep.GEMMS) == sorted(o for o in ops if o.startswith("fc"))
+    M, H, F = bench.layer_dims()
+    assert (M, H, F) == (8192, 4096, 16384)
+    assert 6 * 2 * M * H * F == 6597069766656

@@ -20,29 +20,58 @@ def _quant_gpu(x_dev):
     return host(t.q), host(t.s)
 
 
-@pytest.mark.parametrize("path", ["tma", "plain"])
-@pytest.mark.parametrize("shape", [(32, 32), (96, 160), (256, 256), (64, 4096), (544, 96)])
-@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
-def test_quantize_bit_exact(shape, dtype, path, monkeypatch):
-    """Both quantizer kernels: TMA-staged tiles (the default) and plain loads (JF_PLAIN_LOADS=1),
-    including odd block-column counts (the last tile's second block lies past the last column)."""
-    if path == "plain":
-        monkeypatch.setenv("JF_PLAIN_LOADS", "1")
+QUANT_SHAPES = [(32, 32), (96, 160), (256, 256), (64, 4096), (544, 96)]
+ROWSTATS_SHAPES = [(32, 32), (96, 160), (64, 4096), (544, 96)]
+DTYPES = ["f32", "bf16", "f16"]
+
+
+def _device_input(x, dtype):
+    if dtype == "f32":
+        return dev_f32(x), x
+    if dtype == "bf16":
+        bits = S.to_bf16_bits(x)
+        return dev_bf16(bits), O.bf16_bits_to_f32(bits)
+    h = S.to_f16(x)
+    return torch.from_numpy(h).cuda(), h.astype(np.float32)
+
+
+def check_quantize(shape, dtype):
     rng = np.random.default_rng(zlib.crc32(f"{shape} {dtype}".encode()))  # stable across processes
     x = S.activation(rng, shape[0], shape[1], max(1, shape[1] // 100), 100.0)
-    if dtype == "f32":
-        xd, xh = dev_f32(x), x
-    elif dtype == "bf16":
-        bits = S.to_bf16_bits(x)
-        xd, xh = dev_bf16(bits), O.bf16_bits_to_f32(bits)
-    else:
-        h = S.to_f16(x)
-        xd, xh = torch.from_numpy(h).cuda(), h.astype(np.float32)
+    xd, xh = _device_input(x, dtype)
     q, s = _quant_gpu(xd)
     qr, sr = O.quantize_block(xh)
     check_status()
-    assert np.array_equal(s, sr)
-    assert np.array_equal(q, qr)
+    assert np.array_equal(s, sr), f"{shape} {dtype}"
+    assert np.array_equal(q, qr), f"{shape} {dtype}"
+
+
+@pytest.mark.parametrize("shape", QUANT_SHAPES)
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_quantize_bit_exact(shape, dtype):
+    """The TMA-staged quantizer (the default kernel), including odd block-column counts (the last
+    tile's second block lies past the last column)."""
+    check_quantize(shape, dtype)
+
+
+def test_quantize_plain_load_kernel():
+    """The plain-load quantizer kernel, which the library selects for every call when JF_PLAIN_LOADS=1
+    is in the environment as it loads: a child process with that setting runs the bit-exactness cases
+    of both quantizer entry points (codes, scales and row statistics)."""
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    code = ("import sys; sys.path[:0] = [%r, %r]\n"
+            "import test_gpu_blockwise as T\n"
+            "for shp in T.QUANT_SHAPES:\n"
+            "    for dt in T.DTYPES: T.check_quantize(shp, dt)\n"
+            "for shp in T.ROWSTATS_SHAPES:\n"
+            "    for dt in T.DTYPES: T.check_rowstats(shp, dt)\n"
+            "print('plain-load cases ok')\n") % (here, os.path.dirname(here))
+    res = subprocess.run([sys.executable, "-c", code], env={**os.environ, "JF_PLAIN_LOADS": "1"},
+                         capture_output=True, text=True, timeout=600)
+    assert res.returncode == 0 and "plain-load cases ok" in res.stdout, res.stdout[-2000:] + res.stderr[-4000:]
 
 
 def test_quantize_adversarial_and_ties():
@@ -226,30 +255,25 @@ def test_empty_inputs_are_noops():
 # --------------------------------------------------------------------------------------------
 # f1, second half: the quantizer hands LayerNorm_i8 its row statistics
 # --------------------------------------------------------------------------------------------
-@pytest.mark.parametrize("path", ["tma", "plain"])
-@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
-@pytest.mark.parametrize("shape", [(32, 32), (96, 160), (64, 4096), (544, 96)])
-def test_quantize_rowstats_bit_exact(shape, dtype, path, monkeypatch):
-    """Codes and scales equal jf_quantize_block's and the oracle's; the per-row, per-block sums of q
-    and q^2 equal the oracle's exactly, on both quantizer kernels and odd block-column counts."""
-    if path == "plain":
-        monkeypatch.setenv("JF_PLAIN_LOADS", "1")
+def check_rowstats(shape, dtype):
     rng = np.random.default_rng(zlib.crc32(f"rowstats {shape} {dtype}".encode()))
     x = S.activation(rng, shape[0], shape[1], max(1, shape[1] // 100), 60.0)
     x[5, :] = 0.0
-    if dtype == "f32":
-        xd, xh = dev_f32(x), x
-    elif dtype == "bf16":
-        bits = S.to_bf16_bits(x)
-        xd, xh = dev_bf16(bits), O.bf16_bits_to_f32(bits)
-    else:
-        h = S.to_f16(x)
-        xd, xh = torch.from_numpy(h).cuda(), h.astype(np.float32)
+    xd, xh = _device_input(x, dtype)
     t, st = jf.quantize_block_rowstats(xd)
     qr, sr, str_ = O.quantize_block_rowstats(xh)
     check_status()
-    assert np.array_equal(host(t.q), qr) and np.array_equal(host(t.s), sr)
-    assert np.array_equal(host(st).astype(np.int64), str_)
+    assert np.array_equal(host(t.q), qr) and np.array_equal(host(t.s), sr), f"{shape} {dtype}"
+    assert np.array_equal(host(st).astype(np.int64), str_), f"{shape} {dtype}"
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("shape", ROWSTATS_SHAPES)
+def test_quantize_rowstats_bit_exact(shape, dtype):
+    """Codes and scales equal jf_quantize_block's and the oracle's; the per-row, per-block sums of q
+    and q^2 equal the oracle's exactly, on odd block-column counts too (the plain-load kernel is
+    checked by test_quantize_plain_load_kernel)."""
+    check_rowstats(shape, dtype)
 
 
 @pytest.mark.parametrize("M,H", [(32, 32), (64, 1024), (96, 4096), (32, 6144), (8192, 4096)])

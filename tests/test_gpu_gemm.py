@@ -184,3 +184,21 @@ def test_gemm_hidden4096_sampled(name, mode):
     # the re-quantization of every block is the quantizer rule applied to the fp32 result
     qq, ss = O.quantize_block(y)
     assert np.array_equal(q, qq) and np.array_equal(s, ss)
+
+
+# ----------------------------------------------------------------- plain INT8 product (tensor ceiling)
+@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (384, 512, 1024), (256, 768, 4096)])
+def test_plain_int8_gemm_exact(M, N, K):
+    """jf_gemm_i8_s32, the unscaled INT8 product the bench uses as the measured tensor-core
+    ceiling: exact against the int64 product, including the extreme codes -128 and 127."""
+    rng = np.random.default_rng(M + N + K)
+    a = rng.integers(-128, 128, size=(M, K)).astype(np.int8)
+    b = rng.integers(-128, 128, size=(N, K)).astype(np.int8)
+    a[0, :] = -128
+    b[0, :] = -128
+    b[1, :] = 127
+    c = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    jf.jf_gemm_i8_s32(torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda(), c)
+    ref = a.astype(np.int64) @ b.astype(np.int64).T
+    assert np.array_equal(host(c).astype(np.int64), ref)
+    check_status()
