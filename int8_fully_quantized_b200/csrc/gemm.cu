@@ -10,31 +10,42 @@
 //
 // Design of the block-scaled kernel (one CTA per SM, persistent over 128 x 128 output tiles). The
 // rescale needs, per output element and contraction block, an int32 -> fp32 conversion and an FMA
-// on the CUDA cores, four times the tensor core's time for the same block, so the kernel is built
-// to keep the epilogue warps busy without pause; the tensor core only has to stay ahead of them.
-// Each contraction block of a tile is one MMA into its own int32 TMEM accumulator; four such
+// on the CUDA cores, several times the tensor core's time for the same block, so the kernel is
+// built to keep the epilogue warps busy; the tensor core only has to stay ahead of them. Each
+// contraction block of a tile is one MMA into its own int32 TMEM accumulator; four such
 // accumulators (all 512 TMEM columns) rotate, so the MMAs run up to four blocks ahead:
 //   warp 0       producer: lane 0 loads 128-byte-deep stages of A and B (TMA, 128-byte swizzle,
 //                no multicast) into a 6-stage shared-memory ring; a slot is refilled once the MMAs
 //                that read it have completed (tcgen05.commit on the slot's `empty` barrier).
-//   warp 1       MMA: lane 0 issues one tcgen05.mma (M=128, N=128, K=32) per contraction block and
-//                commits it to that accumulator's `tfull` barrier. It reuses accumulator b as soon
-//                as all 8 epilogue warps have read it: they each bar.arrive on hardware barrier
-//                1 + b after their TMEM load, and warp 1 waits there with bar.sync (the only
-//                thread that waits on that hand-off), so no epilogue warp ever stalls on a release.
-//   warps 2-9    epilogue: warp w owns TMEM lanes 32 (w % 4) .. +31 and two 32-column blocks, i.e.
-//                two 32x32 output blocks of the tile. Per contraction block it waits for the
-//                accumulator's commit, loads its 64 int32 partials per thread (one tcgen05.ld),
-//                arrives on the hand-off barrier, and accumulates fp32(sA*sB) * P in registers
-//                (packed fma.rn.f32x2). The block scales come from global memory straight into
-//                registers, 32 contraction blocks per load (lane l holds block w0 + l), one window
-//                ahead, and are broadcast by warp shuffles. After the last block the warp reduces
-//                each block's absmax and writes its 32x32 codes, the block scale and (optionally)
-//                the fp32 result. Ten warps in all keep at most three on an SM sub-partition, so
-//                each thread may hold the 64 accumulators and 64 partials in registers.
+//   warps 1-2    MMA: warp 1 + m issues the MMAs (M=128, N=128, K=32, one per contraction block)
+//                of pipeline stages m, m + 2, ..., each committed to its accumulator's `tfull`
+//                barrier. It reuses accumulator b as soon as all epilogue warps have read it:
+//                they each bar.arrive on a hand-off hardware barrier after their TMEM load and the
+//                MMA warp waits there with bar.sync. Two warps alternate stages because a lone
+//                thread issues at most about one MMA per ~220 cycles.
+//   warps 3-10   epilogue: warp w owns TMEM lanes 32 (w % 4) .. +31 and two 32-column blocks, i.e.
+//                two 32x32 output blocks of the tile. Per contraction block it waits (bar.sync)
+//                for the watcher's signal, loads its 64 int32 partials per thread (one tcgen05.ld),
+//                arrives on the hand-off barrier, and accumulates fp32(sA*sB) * P in registers.
+//                The block scales come from global memory straight into registers, 32 contraction
+//                blocks per load (lane l holds block w0 + l), one window ahead, and are broadcast
+//                by warp shuffles. After the last block the warp reduces each block's absmax and
+//                writes its 32x32 codes, the block scale and (optionally) the fp32 result.
+//   warp 11      completion watcher: lane 0 is the only thread that polls the `tfull` mbarriers;
+//                once block g's MMA has completed it releases the epilogue warps through hardware
+//                barrier 9 + g % 4. Measured on B200: with all 256 epilogue threads polling the
+//                mbarriers instead, the MMA issue and commit latencies grew several-fold and the
+//                kernel ran ~35% slower.
+// Twelve warps keep at most three on an SM sub-partition, so each thread may hold 64 accumulators
+// and 64 partials in registers.
 // Operand orientation: A and B are read K-major (contraction contiguous) or MN-major (output
 // index contiguous) straight from their row-major INT8 storage, so dgrad and wgrad re-block along
 // the other axis with no transpose pass.
+//
+// Ordering of the hand-offs: an accumulator is handed back only after tcgen05.wait::ld has returned
+// (its partials are in registers), and it is read only after its MMA's commit has been observed on
+// the mbarrier, so the barrier instructions themselves order the TMEM accesses; no tcgen05 fence is
+// issued per contraction block (only around the TMEM allocation and release).
 //
 // Every mbarrier wait is bounded (ptx.cuh). On a timeout the warp that saw it sets the CTA's abort
 // flag; every warp then stops waiting and computing but keeps its place in the hardware-barrier
@@ -60,9 +71,12 @@ constexpr int KB = 32;              // contraction block (one MMA, one rescale)
 constexpr int KBS = 4;              // contraction blocks per pipeline stage (128 bytes)
 constexpr int NBUF = 4;             // TMEM accumulators (4 x 128 = all 512 columns)
 constexpr int STAGES = 6;
+constexpr int NUM_MMA_WARPS = 2;    // alternate pipeline stages
+constexpr int FIRST_EPI_WARP = 1 + NUM_MMA_WARPS;
 constexpr int NUM_EPI_WARPS = 8;    // each owns two 32x32 output blocks of the 128 x 128 tile
-constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
-constexpr uint32_t HANDOFF_THREADS = 32 * (NUM_EPI_WARPS + 1);   // epilogue warps + the MMA warp
+constexpr int WATCH_WARP = FIRST_EPI_WARP + NUM_EPI_WARPS;   // relays MMA completions to the epilogue
+constexpr int NUM_THREADS = 32 * (WATCH_WARP + 1);
+constexpr uint32_t HANDOFF_THREADS = 32 * (NUM_EPI_WARPS + 1);   // epilogue warps + one MMA warp
 constexpr int A_STAGE = BM * KBS * KB;  // 16 KB
 constexpr int B_STAGE = BN * KBS * KB;  // 16 KB
 constexpr uint32_t TMEM_COLS = NBUF * BN;
@@ -70,7 +84,7 @@ constexpr uint32_t TMEM_COLS = NBUF * BN;
 constexpr int SMEM_A = 0;
 constexpr int SMEM_B = SMEM_A + STAGES * A_STAGE;
 constexpr int SMEM_BAR = SMEM_B + STAGES * B_STAGE;
-constexpr int NUM_BARS = 2 * STAGES + NBUF + 1;
+constexpr int NUM_BARS = 2 * STAGES + NBUF + NUM_MMA_WARPS;
 constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
 constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;  // + slack to align the base to 1024
 
@@ -150,7 +164,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_co
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < NBUF; ++b) mbar_init(&tfull[b], 1);
-    mbar_init(drain, 1);
+    for (int m = 0; m < NUM_MMA_WARPS; ++m) mbar_init(&drain[m], 1);
     *abort_flag = 0u;
     fence_mbar_init();
   }
@@ -200,63 +214,85 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_co
         if (pending & (1u << s)) mbar_wait_teardown(&full[s], (pend_ph >> s) & 1u, p.status);
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA warp
+  } else if (warp < FIRST_EPI_WARP) {
+    // ------------------------------------------------------------------ MMA warps
+    // Warp 1 + m issues the MMAs of the CTA's pipeline stages s = m, m + 2, ... (each stage's four
+    // contraction blocks, in order). Before the MMA of contraction block G (G >= NBUF) it waits on
+    // hardware barrier hand_bar(G) until every epilogue warp has read accumulator G % NBUF, i.e.
+    // block G - NBUF. The two warps use disjoint barriers, so each barrier's phases are only ever
+    // waited on by one warp, in order; each warp commits its own stages' `empty` barriers.
     constexpr uint32_t idesc = instr_desc<A_MN, B_MN, BN>();
-    // Position of the next contraction block to issue: tile-local block kb of the CTA's stage seq.
-    int it_kb = 0, it_stage = 0;
+    const int m = warp - 1;
     bool dead = false, issued = false;
-    // Issue the MMA of the next contraction block (in order) into accumulator `buf` (lane 0 only).
-    auto issue_next = [&](uint32_t buf) -> bool {
-      const int ks = it_kb / KBS, kk = it_kb % KBS;
-      const int slot = it_stage % STAGES;
-      if (kk == 0) {
-        if (!mbar_wait(&full[slot], uint32_t(it_stage / STAGES) & 1u, abort_flag, p.status)) return false;
-        tc_fence_after();
-      }
-      const uint32_t a_addr = smem_u32(sA + slot * A_STAGE);
-      const uint32_t b_addr = smem_u32(sB + slot * B_STAGE);
-      // K-major: the 32-byte K step moves inside the 128-byte swizzle row;
-      // MN-major: it moves by 32 rows of 128 bytes (four 8-row swizzle atoms).
-      const uint64_t ad = smem_desc(a_addr + (A_MN ? kk * 4096 : kk * 32), A_MN ? 16384 : 16, 1024);
-      const uint64_t bd = smem_desc(b_addr + (B_MN ? kk * 4096 : kk * 32), B_MN ? 16384 : 16, 1024);
-      mma_i8(tmem_base + buf * BN, ad, bd, idesc, 0u);
-      tc_commit(&tfull[buf]);
-      issued = true;
+    for (int s = m; s < total_stages; s += NUM_MMA_WARPS) {
+      const int ks = s % num_kstages;
+      const int g0 = (s / num_kstages) * kblocks + ks * KBS;
       const int nk = min(KBS, kblocks - ks * KBS);
-      if (kk == nk - 1) {
-        tc_commit(&empty[slot]);   // the stage's last MMA: the slot may be refilled once it completes
-        ++it_stage;
+      const int slot = s % STAGES;
+      for (int kk = 0; kk < nk; ++kk) {
+        const int G = g0 + kk;
+        const uint32_t b = uint32_t(G) & (NBUF - 1);
+        if (G >= NBUF) named_bar_sync(1 + b + NBUF * m, HANDOFF_THREADS);   // block G - NBUF was read
+        if (lane == 0) {
+          if (kk == 0 && !dead) dead = !mbar_wait(&full[slot], uint32_t(s / STAGES) & 1u, abort_flag, p.status);
+          // after a timeout every block's barrier is still completed (plain arrive), so the watcher
+          // and the epilogue keep their order and finish
+          if (dead) mbar_arrive(&tfull[b]);
+          if (!dead) {
+            const uint32_t a_addr = smem_u32(sA + slot * A_STAGE);
+            const uint32_t b_addr = smem_u32(sB + slot * B_STAGE);
+            // K-major: the 32-byte K step moves inside the 128-byte swizzle row;
+            // MN-major: it moves by 32 rows of 128 bytes (four 8-row swizzle atoms).
+            const uint64_t ad = smem_desc(a_addr + (A_MN ? kk * 4096 : kk * 32), A_MN ? 16384 : 16, 1024);
+            const uint64_t bd = smem_desc(b_addr + (B_MN ? kk * 4096 : kk * 32), B_MN ? 16384 : 16, 1024);
+            mma_i8(tmem_base + b * BN, ad, bd, idesc, 0u);
+            tc_commit(&tfull[b]);
+            issued = true;
+          }
+        }
+        __syncwarp();
       }
-      if (++it_kb == kblocks) it_kb = 0;
-      return true;
-    };
-    if (lane == 0) {
-      for (int g = 0; g < min(NBUF, total) && !dead; ++g) dead = !issue_next(uint32_t(g));
-    }
-    for (int g = 0; g < total; ++g) {
-      const uint32_t b = uint32_t(g) & (NBUF - 1);
-      named_bar_sync(1 + b, HANDOFF_THREADS);   // every epilogue warp has read accumulator b
-      if (lane == 0 && !dead && g + NBUF < total) {
-        tc_fence_after();
-        dead = !issue_next(b);
-      }
+      if (lane == 0 && !dead) tc_commit(&empty[slot]);   // the slot may be refilled once these MMAs complete
       __syncwarp();
     }
+    // The last NBUF hand-offs precede no MMA; warp 1 takes them so that every phase completes.
+    if (m == 0)
+      for (int G = max(total, NBUF); G < total + NBUF; ++G) named_bar_sync(1 + (uint32_t(G) & (NBUF - 1)), HANDOFF_THREADS);
     // Teardown: no MMA may still be writing TMEM when it is freed.
     if (lane == 0 && issued) {
-      tc_commit(drain);
-      mbar_wait_teardown(drain, 0u, p.status);
+      tc_commit(&drain[m]);
+      mbar_wait_teardown(&drain[m], 0u, p.status);
     }
     __syncwarp();
+  } else if (warp == WATCH_WARP) {
+    // ------------------------------------------------------------------ completion watcher
+    // The only thread that polls the accumulators' mbarriers: once block g's MMA has completed it
+    // releases the epilogue warps through hardware barrier 9 + g % NBUF (they wait there with
+    // bar.sync, without polling).
+    // Every block's barrier completes, by its MMA's commit or, after a timeout elsewhere, by the MMA
+    // warp's plain arrive, so this wait ignores the abort flag; its limit (three watchdog periods)
+    // outlasts every other bounded wait. Should it still run out, the watcher waits on the release
+    // barrier itself (bar.sync) from then on, so it never runs ahead of the epilogue warps.
+    uint32_t never = 0u;
+    bool lost = false;
+    for (int g = 0; g < total; ++g) {
+      const uint32_t b = uint32_t(g) & (NBUF - 1);
+      bool good = true;
+      if (lane == 0 && !lost) {
+        const uint32_t ph = uint32_t(g / NBUF) & 1u;
+        good = mbar_try_wait(&tfull[b], ph) || mbar_wait(&tfull[b], ph, &never, p.status, 3 * kWatchdogNs);
+      }
+      lost = lost || !__shfl_sync(0xffffffffu, good, 0);
+      if (lost) named_bar_sync(9 + b, HANDOFF_THREADS);
+      else named_bar_arrive(9 + b, HANDOFF_THREADS);
+    }
   } else {
     // ------------------------------------------------------------------ epilogue warps
     const int sub = warp & 3;             // TMEM sub-partition this warp may access = row block in the tile
-    const int cb0 = ((warp - 2) >> 2) * 2;  // first of the warp's two column blocks in the tile
+    const int cb0 = ((warp - FIRST_EPI_WARP) >> 2) * 2;  // first of the warp's two column blocks in the tile
     const uint32_t t_base = tmem_base + (uint32_t(sub * 32) << 16) + uint32_t(cb0 * 32);
     const int nrb = p.rows >> 5, ncb = p.cols >> 5;
-    bool dead = false;
-    uint32_t g = 0;                       // contraction blocks consumed so far (accumulator g % NBUF)
+    const bool whole_stages = (kblocks % KBS) == 0;   // then every stage holds KBS blocks
     // Scales of the current window (lane l: contraction block w0 + l) of the warp's row block (sa)
     // and two column blocks (sb0, sb1); each window prefetches the next one.
     float sa_n, sb0_n, sb1_n;
@@ -267,6 +303,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_co
       sb1_n = scale_window(p.b_s, p.b_s_blk, p.b_s_k, cbk + 1, valid ? ncb : 0, w0, kblocks, lane);
     };
     load_scales(blockIdx.x, 0, my_tiles > 0);
+    int g = 0;                            // contraction blocks consumed so far (accumulator g % NBUF)
     for (int tile = 0; tile < my_tiles; ++tile) {
       const int t = blockIdx.x + tile * gridDim.x;
       const int rbk = (t % p.tiles_m) * (BM / 32) + sub, cbk = (t / p.tiles_m) * (BN / 32) + cb0;
@@ -279,32 +316,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_co
         else load_scales(t + gridDim.x, 0, tile + 1 < my_tiles);  // the start of the next one
         const int nk = min(32, kblocks - w0);
         for (int j = 0; j < nk; ++j, ++g) {
-          const uint32_t b = g & (NBUF - 1);
-          dead = dead || __any_sync(0xffffffffu, *abort_flag != 0u);
+          const uint32_t b = uint32_t(g) & (NBUF - 1);
           uint32_t r[64];
-          if (!dead) {
-            const uint32_t ph = (g / NBUF) & 1u;
-            const bool good = mbar_try_wait(&tfull[b], ph) || mbar_wait(&tfull[b], ph, abort_flag, p.status);
-            dead = !__all_sync(0xffffffffu, good);
+          named_bar_sync(9 + b, HANDOFF_THREADS);   // the watcher saw block g's MMA complete
+          tmem_ld_32x32b_x64(t_base + b * BN, r);
+          tc_wait_ld64(r);   // the partials are in registers: the MMA may overwrite the accumulator
+          {  // hand accumulator b back: the barrier of the MMA warp of block g + NBUF (the warp of that
+             // block's stage; warp 1 takes the hand-offs past the last block)
+            const int G = g + NBUF;
+            int sn = 0;
+            if (G < total) {
+              if (whole_stages) {
+                sn = G / KBS;
+              } else {
+                const int kn = w0 + j + NBUF;   // tile-local index of block G
+                sn = kn < kblocks ? tile * num_kstages + kn / KBS : (G / kblocks) * num_kstages + (G % kblocks) / KBS;
+              }
+            }
+            named_bar_arrive(1 + b + NBUF * uint32_t(sn % NUM_MMA_WARPS), HANDOFF_THREADS);
           }
-          if (!dead) {
-            tc_fence_after();
-            tmem_ld_32x32b_x64(t_base + b * BN, r);
-            tc_wait_ld64(r);
-          }
-          tc_fence_before();
-          named_bar_arrive(1 + b, HANDOFF_THREADS);   // accumulator b may be reused
           // fp32(sA * sB) of contraction block w0 + j for the warp's two output blocks
           const float a = __shfl_sync(0xffffffffu, sa, j);
           const float c0 = a * __shfl_sync(0xffffffffu, sb0, j), c1 = a * __shfl_sync(0xffffffffu, sb1, j);
-          if (!dead) {
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-              fma_x2(c0, c0, __int2float_rn(int(r[i])), __int2float_rn(int(r[i + 1])), acc[0][i], acc[0][i + 1],
-                     acc[0][i], acc[0][i + 1]);
-              fma_x2(c1, c1, __int2float_rn(int(r[32 + i])), __int2float_rn(int(r[33 + i])), acc[1][i],
-                     acc[1][i + 1], acc[1][i], acc[1][i + 1]);
-            }
+          for (int i = 0; i < 32; i += 2) {   // packed fp32x2 FMAs, each lane rounded as the scalar fmaf
+            fma_x2(c0, c0, __int2float_rn(int(r[i])), __int2float_rn(int(r[i + 1])), acc[0][i], acc[0][i + 1],
+                   acc[0][i], acc[0][i + 1]);
+            fma_x2(c1, c1, __int2float_rn(int(r[32 + i])), __int2float_rn(int(r[33 + i])), acc[1][i], acc[1][i + 1],
+                   acc[1][i], acc[1][i + 1]);
           }
         }
       }
@@ -313,7 +352,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_co
       // unrolled so that acc stays in registers)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        if (dead || rbk >= nrb || cbk + h >= ncb) continue;
+        if (rbk >= nrb || cbk + h >= ncb) continue;
         float (&y)[32] = acc[h];
         const int64_t off = (int64_t(rbk) * 32 + lane) * p.ld_y + int64_t(cbk + h) * 32;
         const int64_t soff = int64_t(rbk) * ncb + cbk + h;
@@ -435,11 +474,9 @@ __global__ void __launch_bounds__(S32_THREADS, 1) gemm_i8_s32_kernel(const __gri
       for (int i = 0; ok && i < my_tiles; ++i) {
         const uint32_t buf = uint32_t(i) & 1u;
         if (!mbar_wait(&tempty[buf], (uint32_t(i >> 1) & 1u) ^ 1u, abort_flag, p.status)) break;
-        tc_fence_after();
         for (int ks = 0; ks < num_kstages; ++ks, ++g) {
           const int st = g % S32_STAGES;
           if (!mbar_wait(&full[st], uint32_t(g / S32_STAGES) & 1u, abort_flag, p.status)) { ok = false; break; }
-          tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + st * S32_A_STAGE), b_addr = smem_u32(sB + st * S32_B_STAGE);
 #pragma unroll
           for (int kk = 0; kk < KBS; ++kk)
