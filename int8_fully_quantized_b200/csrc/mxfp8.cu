@@ -175,7 +175,6 @@ __global__ void __launch_bounds__(mx::NUM_THREADS, 1) mxf8_gemm_kernel(const __g
   const int num_tiles = p.tiles_m * p.tiles_n;
   const int my_tiles = blockIdx.x < num_tiles ? (num_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
   const int total = my_tiles * nks;
-  const int nkw = p.kblocks >> 2;                // scale words per row (K / 128)
   auto tile_of = [&](int i) { return blockIdx.x + i * gridDim.x; };
 
   if (warp == 0) {

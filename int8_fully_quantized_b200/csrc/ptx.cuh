@@ -49,41 +49,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Non-blocking test: has the phase of parity `parity` of `bar` completed?
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Poll with a back-off: one thread tests the phase, sleeping `sleep_ns` between tests, so that a
-// waiting warp puts almost no load on the shared-memory barrier unit (many threads spinning on
-// mbarriers slow down the tensor-core instructions of the same SM). Bounded like mbar_wait.
-__device__ __forceinline__ bool mbar_poll_sleep(uint64_t* bar, uint32_t parity, volatile uint32_t* abort,
-                                                unsigned int* status, unsigned int sleep_ns = 64,
-                                                unsigned long long limit_ns = kWatchdogNs) {
-  if (mbar_test_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer();
-  for (uint32_t n = 1;; ++n) {
-    __nanosleep(sleep_ns);
-    if (mbar_test_wait(bar, parity)) return true;
-    if ((n & 15u) == 0) {
-      if (*abort) return false;
-      if (globaltimer() - t0 > limit_ns) {
-        *abort = 1u;
-        atomicOr(status, kStatusTimeout);
-        return false;
-      }
-    }
-  }
-}
-
 // Wait for the phase of parity `parity` of `bar` to complete. Bounded: gives up when `abort`
 // becomes nonzero (another thread gave up) or after kWatchdogNs, in which case it raises the
 // timeout bit of *status, sets *abort and returns false.
