@@ -66,6 +66,9 @@ def parse_args():
                    help="oracle sample: this many x this many output blocks of each GEMM")
     p.add_argument("--sweep", action="store_true",
                    help="time the memory-bound kernels on the M x 4096 sweep instead of the step")
+    p.add_argument("--profile-gemm", action="store_true",
+                   help="run the three block-scaled GEMM modes on the GPT2-medium fc1 shapes (M=4096, K=1024, "
+                        "N=4096) --steps times each, L2 flushed before each launch: a small case for ncu captures")
     p.add_argument("--sweep-m", type=int, nargs="*", default=[1024, 8192, 65536])
     p.add_argument("--sweep-ops", nargs="*", default=["quantize_bf16", "dequantize_bf16", "gelu_i8", "layernorm_i8",
                                                       "gelu_i8_bwd", "layernorm_i8_bwd", "fused_fc1",
@@ -981,8 +984,36 @@ def host_q(t):
     return t.q.cpu().numpy(), t.s.cpu().numpy()
 
 
+def run_profile_gemm(args):
+    """fwd, dgrad and wgrad of the GPT2-medium fc1 shapes, each launched --steps times in that order
+    (3 warm-up launches of each first), with the L2 flushed before every launch; prints the median
+    device time of each. A small, fixed launch sequence for profiler captures of the GEMM kernel."""
+    import torch
+    import int8_fully_quantized_b200 as jf
+    torch.cuda.set_device(0)
+    jf.load_library()
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    M, K, N, host = gpt2m_inputs(0)
+    X = jf.quantize_block(torch.from_numpy(host["x"].view(np.int16)).cuda().view(torch.bfloat16))
+    W = jf.quantize_block(torch.from_numpy(host["w"].view(np.int16)).cuda().view(torch.bfloat16))
+    from inputs import synthetic as S
+    dY = jf.quantize_block(torch.from_numpy(S.to_bf16_bits(S.grad(np.random.default_rng(5), M, N)).view(np.int16))
+                           .cuda().view(torch.bfloat16))
+    Y, dX, dW = jf.empty_qtensor(M, N), jf.empty_qtensor(M, K), jf.empty_qtensor(N, K)
+    out = {}
+    for name, fn in (("fwd", lambda: jf.jf_linear_fwd(X, W, Y)), ("dgrad", lambda: jf.jf_linear_dgrad(dY, W, dX)),
+                     ("wgrad", lambda: jf.jf_linear_wgrad(dY, X, dW))):
+        ms = _device_ms(fn, flush, reps=max(1, args.steps))
+        out[name] = {"ms": round(ms, 4), "TOPS": round(2 * M * N * K / (ms * 1e-3) / 1e12, 1)}
+    assert jf.jf_device_status() == 0
+    print(json.dumps({"profile_gemm": out, "M": M, "K": K, "N": N}), flush=True)
+
+
 def main():
     args = parse_args()
+    if args.profile_gemm:
+        run_profile_gemm(args)
+        return
     if args.configs:
         run_configs(args)
         return
