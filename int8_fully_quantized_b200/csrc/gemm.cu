@@ -8,7 +8,8 @@
 // exact int32 partial P = sum_k A(r,k) B(c,k) is multiplied by c = fp32(sA(r/32,kb) * sB(c/32,kb))
 // and accumulated in fp32; after the last block the fp32 tile is re-quantized per 32x32 block.
 //
-// Design of the block-scaled kernel (one CTA per SM, persistent over 128 x 128 output tiles). The
+// Design of the block-scaled kernel (one CTA per SM, persistent over 128 x 128 output tiles, in the
+// order that keeps the smaller operand resident in L2: see tile_of). The
 // rescale needs, per output element and contraction block, an int32 -> fp32 conversion and an FMA
 // on the CUDA cores, several times the tensor core's time for the same block, so the kernel is
 // built to keep the epilogue warps busy; the tensor core only has to stay ahead of them. Each
@@ -105,7 +106,16 @@ struct __align__(64) GemmParams {
   unsigned int* status;
   int rows, cols, kblocks;
   int tiles_m, tiles_n;
+  int n_fast;   // tile order: 0 = row tiles vary fastest, 1 = column tiles vary fastest
 };
+
+// Row and column tile of the CTA's tile t. The 148 tiles in flight at once share one operand's
+// blocks: with row tiles varying fastest they cover nearly all row tiles (all of A) and a few
+// column tiles, so A is re-read from L2 by every wave and B streams once; the host picks the order
+// that keeps the smaller operand the re-read one, so that it stays in L2.
+__device__ __forceinline__ int2 tile_of(const GemmParams& p, int t) {
+  return p.n_fast ? make_int2(t / p.tiles_n, t % p.tiles_n) : make_int2(t % p.tiles_m, t / p.tiles_m);
+}
 
 // tcgen05 instruction descriptor: s32 accumulator, signed int8 A and B, A/B major-ness, N, M.
 template <bool A_MN, bool B_MN, int N>
@@ -196,7 +206,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_co
       for (int g = 0; g < total_stages; ++g) {
         const int t = blockIdx.x + (g / num_kstages) * gridDim.x;
         const int ks = g % num_kstages;
-        const int row0 = (t % p.tiles_m) * BM, col0 = (t / p.tiles_m) * BN;
+        const int2 tc = tile_of(p, t);
+        const int row0 = tc.x * BM, col0 = tc.y * BN;
         const int st = g % STAGES;
         const uint32_t ph = uint32_t(g / STAGES) & 1u;
         if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status)) break;
@@ -297,7 +308,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_co
     // and two column blocks (sb0, sb1); each window prefetches the next one.
     float sa_n, sb0_n, sb1_n;
     auto load_scales = [&](int t, int w0, bool valid) {
-      const int rbk = (t % p.tiles_m) * (BM / 32) + sub, cbk = (t / p.tiles_m) * (BN / 32) + cb0;
+      const int2 tc = tile_of(p, t);
+      const int rbk = tc.x * (BM / 32) + sub, cbk = tc.y * (BN / 32) + cb0;
       sa_n = scale_window(p.a_s, p.a_s_blk, p.a_s_k, rbk, valid ? nrb : 0, w0, kblocks, lane);
       sb0_n = scale_window(p.b_s, p.b_s_blk, p.b_s_k, cbk, valid ? ncb : 0, w0, kblocks, lane);
       sb1_n = scale_window(p.b_s, p.b_s_blk, p.b_s_k, cbk + 1, valid ? ncb : 0, w0, kblocks, lane);
@@ -306,7 +318,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_co
     int g = 0;                            // contraction blocks consumed so far (accumulator g % NBUF)
     for (int tile = 0; tile < my_tiles; ++tile) {
       const int t = blockIdx.x + tile * gridDim.x;
-      const int rbk = (t % p.tiles_m) * (BM / 32) + sub, cbk = (t / p.tiles_m) * (BN / 32) + cb0;
+      const int2 tc = tile_of(p, t);
+      const int rbk = tc.x * (BM / 32) + sub, cbk = tc.y * (BN / 32) + cb0;
       float acc[2][32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) acc[0][i] = acc[1][i] = 0.0f;
@@ -614,6 +627,7 @@ cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t st) {
   prm.cols = int(g.cols);
   prm.kblocks = int(kbn);
   prm.tiles_m = int((g.rows + BM - 1) / BM);
+  prm.n_fast = g.rows > g.cols ? 1 : 0;   // A (rows x depth) larger than B: keep B in L2
   prm.tiles_n = int((g.cols + BN - 1) / BN);
   const int tiles = prm.tiles_m * prm.tiles_n;
   const int grid = tiles < sm_count ? tiles : sm_count;
