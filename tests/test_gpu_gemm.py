@@ -52,6 +52,8 @@ SHAPES = [
     (352, 544, 416),   # 3 x 3 tiles with ragged edges, 13 contraction blocks (ragged stage)
     (256, 256, 256),   # the single-linear workload
     (224, 1024, 1056),
+    (544, 352, 416),   # more rows than columns: the column tiles vary fastest
+    (1056, 224, 96),   # the same with three contraction blocks (one partial stage)
 ]
 
 
