@@ -222,7 +222,7 @@ class GpuStep:
         import torch
         import int8_fully_quantized_b200 as jf
         self.jf, self.torch = jf, torch
-        M, H, F = layer_dims()
+        (M, H), F = host["x"].shape, host["w1"].shape[0]   # the layer's sizes, from its inputs
         self.M, self.H, self.F, self.world = M, H, F, world_size
         dev = torch.device("cuda", torch.cuda.current_device())
         bf = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
