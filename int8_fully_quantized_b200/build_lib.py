@@ -19,6 +19,9 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libjetfire.so")
 HASH_PATH = LIB_PATH + ".srchash"
+# The same sources with NVTX ranges around every compute entry point (-DJF_NVTX), for profiling with
+# a tool that records NVTX; load it with JETFIRE_LIB=<this path>. The product library has no ranges.
+NVTX_LIB_PATH = os.path.join(PKG_DIR, "libjetfire_nvtx.so")
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
@@ -98,6 +101,22 @@ def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | N
     return LIB_PATH
 
 
+def build_nvtx(verbose: bool = False) -> str:
+    """Compile the instrumented variant (NVTX ranges, -DJF_NVTX) into ``libjetfire_nvtx.so``."""
+    tmp = NVTX_LIB_PATH + ".tmp"
+    cmd = [_nvcc(), *ARCH_FLAGS, *NVCC_FLAGS, "-DJF_NVTX", "-I", INCLUDE, "-I", CSRC, *sources(), "-o", tmp]
+    if verbose:
+        print(" ".join(cmd), file=sys.stderr)
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
+    os.replace(tmp, NVTX_LIB_PATH)
+    return NVTX_LIB_PATH
+
+
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True,
-                extra_flags=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None))
+    if "--nvtx" in sys.argv:
+        print(build_nvtx(verbose=True))
+    else:
+        print(build(force="--force" in sys.argv, verbose=True,
+                    extra_flags=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None))

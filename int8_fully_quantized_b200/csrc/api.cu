@@ -4,6 +4,21 @@
 #include <mutex>
 #include <cuda_runtime.h>
 
+// NVTX ranges around the compute entry points, compiled in only with -DJF_NVTX (the separate
+// instrumented build of build_lib.py --nvtx): header-only NVTX 3, no library to link.
+#ifdef JF_NVTX
+#include <nvtx3/nvToolsExt.h>
+namespace {
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+}  // namespace
+#define JF_RANGE(name) const NvtxRange jf_nvtx_range_(name)
+#else
+#define JF_RANGE(name) ((void)0)
+#endif
+
 #include "jetfire.h"
 #include "kernels.h"
 #include "ptx.cuh"
@@ -198,16 +213,19 @@ static int quantize_impl(const void* x, jf_dtype dt, int64_t rows, int64_t cols,
 
 int jf_quantize_block(const void* x, jf_dtype dt, int64_t rows, int64_t cols, int8_t* q, float* s,
                       void* stream) {
+  JF_RANGE(__func__);
   return quantize_impl(x, dt, rows, cols, q, s, nullptr, false, stream);
 }
 
 int jf_quantize_block_rowstats(const void* x, jf_dtype dt, int64_t rows, int64_t cols, int8_t* q, float* s,
                                int32_t* stats, void* stream) {
+  JF_RANGE(__func__);
   return quantize_impl(x, dt, rows, cols, q, s, stats, true, stream);
 }
 
 int jf_dequantize_block(const int8_t* q, const float* s, int64_t rows, int64_t cols, void* y, jf_dtype dt,
                         void* stream) {
+  JF_RANGE(__func__);
   if (dt != JF_F32 && dt != JF_BF16 && dt != JF_F16) return JF_ERR_DTYPE;
   if (!dims_ok(rows, cols)) return JF_ERR_SHAPE;
   if (rows == 0 || cols == 0) return JF_OK;
@@ -221,12 +239,14 @@ int jf_dequantize_block(const int8_t* q, const float* s, int64_t rows, int64_t c
 }
 
 int jf_linear_fwd(jf_cqtensor X, jf_cqtensor W, jf_qtensor Y, float* y_f32, void* stream) {
+  JF_RANGE(__func__);
   if (!dims_ok(X.rows, X.cols) || !dims_ok(W.rows, W.cols)) return JF_ERR_SHAPE;
   if (X.cols != W.cols) return JF_ERR_SHAPE;
   return gemm_call(jf::kFwd, X, W, Y, y_f32, X.rows, W.rows, X.cols, stream);
 }
 
 int jf_linear_fwd_gelu(jf_cqtensor X, jf_cqtensor W, jf_qtensor Y, jf_qtensor Ypre, void* stream) {
+  JF_RANGE(__func__);
   if (!dims_ok(X.rows, X.cols) || !dims_ok(W.rows, W.cols)) return JF_ERR_SHAPE;
   if (X.cols != W.cols) return JF_ERR_SHAPE;
   if (Y.q == nullptr && X.rows != 0 && W.rows != 0) return JF_ERR_NULL;
@@ -234,18 +254,21 @@ int jf_linear_fwd_gelu(jf_cqtensor X, jf_cqtensor W, jf_qtensor Y, jf_qtensor Yp
 }
 
 int jf_linear_dgrad(jf_cqtensor dY, jf_cqtensor W, jf_qtensor dX, float* dx_f32, void* stream) {
+  JF_RANGE(__func__);
   if (!dims_ok(dY.rows, dY.cols) || !dims_ok(W.rows, W.cols)) return JF_ERR_SHAPE;
   if (dY.cols != W.rows) return JF_ERR_SHAPE;
   return gemm_call(jf::kDgrad, dY, W, dX, dx_f32, dY.rows, W.cols, dY.cols, stream);
 }
 
 int jf_linear_wgrad(jf_cqtensor dY, jf_cqtensor X, jf_qtensor dW, float* dw_f32, void* stream) {
+  JF_RANGE(__func__);
   if (!dims_ok(dY.rows, dY.cols) || !dims_ok(X.rows, X.cols)) return JF_ERR_SHAPE;
   if (dY.rows != X.rows) return JF_ERR_SHAPE;
   return gemm_call(jf::kWgrad, dY, X, dW, dw_f32, dY.cols, X.cols, dY.rows, stream);
 }
 
 int jf_gelu_i8(jf_cqtensor X, jf_qtensor Y, void* stream) {
+  JF_RANGE(__func__);
   int st;
   if ((st = check_cq(X)) != JF_OK) return st;
   if ((st = check_q(Y, true)) != JF_OK) return st;
@@ -286,15 +309,18 @@ static int layernorm_impl(jf_cqtensor X, const int32_t* stats, bool want_stats, 
 
 int jf_layernorm_i8(jf_cqtensor X, const float* gamma, const float* beta, float eps, jf_qtensor Y,
                     void* stream) {
+  JF_RANGE(__func__);
   return layernorm_impl(X, nullptr, false, gamma, beta, eps, Y, stream);
 }
 
 int jf_layernorm_i8_rowstats(jf_cqtensor X, const int32_t* stats, const float* gamma, const float* beta, float eps,
                              jf_qtensor Y, void* stream) {
+  JF_RANGE(__func__);
   return layernorm_impl(X, stats, true, gamma, beta, eps, Y, stream);
 }
 
 int jf_gelu_i8_bwd(jf_cqtensor X, jf_cqtensor dY, jf_qtensor dX, void* stream) {
+  JF_RANGE(__func__);
   int st;
   if ((st = check_cq(X)) != JF_OK) return st;
   if ((st = check_cq(dY)) != JF_OK) return st;
@@ -364,6 +390,7 @@ extern "C" {
 
 int jf_layernorm_i8_bwd(jf_cqtensor X, jf_cqtensor dY, const float* gamma, float eps, jf_qtensor dX, float* dgamma,
                         float* dbeta, void* workspace, int64_t workspace_bytes, void* stream) {
+  JF_RANGE(__func__);
   int st;
   if ((st = ln_bwd_validate(X, dY, gamma, dX, dgamma, dbeta)) != JF_OK) return st;
   if (X.rows == 0 || X.cols == 0) return JF_OK;
@@ -382,6 +409,7 @@ int jf_layernorm_i8_bwd(jf_cqtensor X, jf_cqtensor dY, const float* gamma, float
 
 int jf_layernorm_i8_bwd_noalloc(jf_cqtensor X, jf_cqtensor dY, const float* gamma, float eps, jf_qtensor dX,
                                 float* dgamma, float* dbeta, void* stream) {
+  JF_RANGE(__func__);
   // the same argument checks, in the same order, as jf_layernorm_i8_bwd; only then the scratch size
   int st;
   if ((st = ln_bwd_validate(X, dY, gamma, dX, dgamma, dbeta)) != JF_OK) return st;
@@ -412,6 +440,7 @@ bool gran_ok(jf_granularity g) { return g == JF_GRAN_BLOCK || g == JF_GRAN_TOKEN
 
 int jf_quantize_granular(const void* x, jf_dtype dt, int64_t rows, int64_t cols, jf_granularity g, int8_t* q,
                          float* s, void* stream) {
+  JF_RANGE(__func__);
   if (dt != JF_F32 && dt != JF_BF16 && dt != JF_F16) return JF_ERR_DTYPE;
   if (!gran_ok(g)) return JF_ERR_ARG;
   if (!dims_ok(rows, cols)) return JF_ERR_SHAPE;
@@ -429,6 +458,7 @@ int jf_quantize_granular(const void* x, jf_dtype dt, int64_t rows, int64_t cols,
 
 int jf_dequantize_granular(const int8_t* q, const float* s, int64_t rows, int64_t cols, jf_granularity g, void* y,
                            jf_dtype dt, void* stream) {
+  JF_RANGE(__func__);
   if (dt != JF_F32 && dt != JF_BF16 && dt != JF_F16) return JF_ERR_DTYPE;
   if (!gran_ok(g)) return JF_ERR_ARG;
   if (!dims_ok(rows, cols)) return JF_ERR_SHAPE;
@@ -445,6 +475,7 @@ int jf_dequantize_granular(const int8_t* q, const float* s, int64_t rows, int64_
 
 int jf_quantization_error(const void* x, jf_dtype dt, const int8_t* q, const float* s, int64_t rows, int64_t cols,
                           jf_granularity g, double* sums, void* stream) {
+  JF_RANGE(__func__);
   if (dt != JF_F32 && dt != JF_BF16 && dt != JF_F16) return JF_ERR_DTYPE;
   if (!gran_ok(g)) return JF_ERR_ARG;
   if (!dims_ok(rows, cols)) return JF_ERR_SHAPE;
@@ -466,6 +497,7 @@ int jf_quantization_error(const void* x, jf_dtype dt, const int8_t* q, const flo
 
 int jf_mx_quantize(const void* x, jf_dtype dt, int64_t rows, int64_t cols, uint8_t* codes, uint8_t* scales,
                    void* stream) {
+  JF_RANGE(__func__);
   if (dt != JF_F32 && dt != JF_BF16 && dt != JF_F16) return JF_ERR_DTYPE;
   if (!dims_ok(rows, cols)) return JF_ERR_SHAPE;
   if (rows == 0 || cols == 0) return JF_OK;
@@ -481,6 +513,7 @@ int jf_mx_quantize(const void* x, jf_dtype dt, int64_t rows, int64_t cols, uint8
 
 int jf_mx_linear_fwd(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes, const uint8_t* b_scales,
                      int64_t M, int64_t N, int64_t K, float* y, void* stream) {
+  JF_RANGE(__func__);
   if (!dims_ok(M, K) || !dims_ok(N, K) || K % 128 != 0) return JF_ERR_SHAPE;
   if (M == 0 || N == 0) return JF_OK;
   if (K == 0) return JF_ERR_SHAPE;
@@ -500,6 +533,7 @@ int jf_mx_linear_fwd(const uint8_t* a_codes, const uint8_t* a_scales, const uint
 }
 
 int jf_gemm_i8_s32(const int8_t* A, const int8_t* B, int32_t* C, int64_t M, int64_t N, int64_t K, void* stream) {
+  JF_RANGE(__func__);
   if (M < 0 || N < 0 || K < 0 || M % 128 != 0 || N % 256 != 0 || K % 128 != 0 || K > 65536 ||
       M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31))
     return JF_ERR_SHAPE;
@@ -516,6 +550,7 @@ int jf_gemm_i8_s32(const int8_t* A, const int8_t* B, int32_t* C, int64_t M, int6
 }
 
 int jf_selftest_wait_timeout(int64_t limit_ns, void* stream) {
+  JF_RANGE(__func__);
   if (limit_ns < 1000000 || limit_ns > 10000000000ll) return JF_ERR_ARG;
   const DevInfo d = device_info();
   if (!d.ok) return JF_ERR_DEVICE;
@@ -541,6 +576,7 @@ const char* jf_strerror(int status) {
 }
 
 int jf_device_status(void* stream) {
+  JF_RANGE(__func__);
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return JF_ERR_CUDA;
   unsigned int v = 0, zero = 0;
   if (cudaMemcpyFromSymbol(&v, jf::g_status, sizeof(v)) != cudaSuccess) return JF_ERR_CUDA;

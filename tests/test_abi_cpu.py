@@ -157,3 +157,17 @@ def test_compute_without_gpu_fails_loudly(lib):
                                            vp(1 << 43), vp(1 << 44), None) == -8
     with pytest.raises(jf.JetfireError):
         jf._check(st, "jf_quantize_block")
+
+
+def test_nvtx_instrumented_entry_points_compile(tmp_path):
+    """The instrumented variant (NVTX ranges around every compute entry point, -DJF_NVTX) compiles;
+    its ranges cover the same entry points the header declares."""
+    src = os.path.join(build_lib.CSRC, "api.cu")
+    with open(src) as f:
+        text = f.read()
+    assert text.count("JF_RANGE(__func__);") >= 20
+    cmd = [build_lib._nvcc(), *build_lib.ARCH_FLAGS, "-O1", "-std=c++17", "-Xcompiler", "-fPIC",
+           "--expt-relaxed-constexpr", "-DJF_NVTX", "-I", build_lib.INCLUDE, "-I", build_lib.CSRC, "-c", src,
+           "-o", str(tmp_path / "api_nvtx.o")]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
