@@ -298,6 +298,8 @@ def quantization_mse(x: torch.Tensor, granularity: str, stream=None) -> float:
     q, s = quantize_granular(x, granularity, stream)
     sums = torch.empty(3, dtype=torch.float64, device=x.device)
     jf_quantization_error(x, q, s, GRANULARITY[granularity], sums, stream)
+    if stream is not None:   # .item() below is ordered after the current stream only
+        stream.synchronize() if hasattr(stream, "synchronize") else torch.cuda.synchronize()
     return float(sums[2].item())
 
 
