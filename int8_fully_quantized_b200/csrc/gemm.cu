@@ -324,7 +324,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_co
 #pragma unroll
       for (int i = 0; i < 32; ++i) acc[0][i] = acc[1][i] = 0.0f;
       for (int w0 = 0; w0 < kblocks; w0 += 32) {
-        const float sa = sa_n, sb0 = sb0_n, sb1 = sb1_n;
+        // lane l: fp32(sA * sB) of contraction block w0 + l for the warp's two output blocks
+        const float cw0 = sa_n * sb0_n, cw1 = sa_n * sb1_n;
         if (w0 + 32 < kblocks) load_scales(t, w0 + 32, true);   // the rest of this tile
         else load_scales(t + gridDim.x, 0, tile + 1 < my_tiles);  // the start of the next one
         const int nk = min(32, kblocks - w0);
@@ -348,9 +349,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_co
             }
             named_bar_arrive(1 + b + NBUF * uint32_t(sn % NUM_MMA_WARPS), HANDOFF_THREADS);
           }
-          // fp32(sA * sB) of contraction block w0 + j for the warp's two output blocks
-          const float a = __shfl_sync(0xffffffffu, sa, j);
-          const float c0 = a * __shfl_sync(0xffffffffu, sb0, j), c1 = a * __shfl_sync(0xffffffffu, sb1, j);
+          const float c0 = __shfl_sync(0xffffffffu, cw0, j), c1 = __shfl_sync(0xffffffffu, cw1, j);
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {   // packed fp32x2 FMAs, each lane rounded as the scalar fmaf
             fma_x2(c0, c0, __int2float_rn(int(r[i])), __int2float_rn(int(r[i + 1])), acc[0][i], acc[0][i + 1],
