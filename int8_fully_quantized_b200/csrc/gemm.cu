@@ -329,6 +329,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_i8_kernel(const __grid_co
         if (w0 + 32 < kblocks) load_scales(t, w0 + 32, true);   // the rest of this tile
         else load_scales(t + gridDim.x, 0, tile + 1 < my_tiles);  // the start of the next one
         const int nk = min(32, kblocks - w0);
+        // two blocks per iteration: measured 7-9% faster than one, bit-identical; four spill registers
+#pragma unroll 2
         for (int j = 0; j < nk; ++j, ++g) {
           const uint32_t b = uint32_t(g) & (NBUF - 1);
           uint32_t r[64];
