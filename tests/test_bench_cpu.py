@@ -50,3 +50,22 @@ def test_step_covers_the_path_and_counts_six_gemms():
     M, H, F = bench.layer_dims()
     assert (M, H, F) == (8192, 4096, 16384)
     assert 6 * 2 * M * H * F == 6597069766656
+
+
+def test_traffic_record_is_reported_only_for_the_sources_it_was_taken_of(tmp_path, monkeypatch):
+    """bench.py reports the dominant GEMM's DRAM traffic from profiles/gemm_traffic.json only while the
+    record's content hash equals that of the current GEMM kernel sources; otherwise null."""
+    import json
+    import os
+    from int8_fully_quantized_b200 import build_lib
+    os.makedirs(tmp_path / "profiles")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    rec = {"fc1_fwd": 211_000_000, "kernel_source_hash": build_lib.kernel_source_hash()}
+    with open(tmp_path / "profiles" / "gemm_traffic.json", "w") as f:
+        json.dump(rec, f)
+    assert bench._load_traffic("fc1_fwd") == 211_000_000
+    assert bench._load_traffic("fc2_fwd") is None          # no figure for that launch
+    rec["kernel_source_hash"] = "0" * 64                      # taken of other sources
+    with open(tmp_path / "profiles" / "gemm_traffic.json", "w") as f:
+        json.dump(rec, f)
+    assert bench._load_traffic("fc1_fwd") is None
